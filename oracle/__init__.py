@@ -1,0 +1,142 @@
+"""CPU oracle for exact attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference leg may import this package. The product library never does.
+
+Two independent routes to the same result:
+
+* :func:`attention` -- the plain definition in fp64 C (``attn_ref.c``): every
+  score row is materialised in full and the softmax is taken in two passes.
+  This follows "FlashAttention (UR)", section "Problem of standard attention".
+* :func:`online.attention_online` -- a blockwise online-softmax evaluation in
+  numpy (running row max and running sum of exponentials, rescaled per key
+  block), following section "Online softmax" of the same page. It exists only
+  so the tests can check that the two evaluation orders agree.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_ref.c")
+_LIB_PATH = os.path.join(_HERE, "_attn_ref.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(src: str = _SRC, out: str = _LIB_PATH, extra_flags=()) -> str:
+    """Compile the oracle with gcc (fp64, OpenMP, no fast-math)."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           *extra_flags, src, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _bind(lib):
+    dp = ctypes.POINTER(ctypes.c_double)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    c_int, c_double = ctypes.c_int, ctypes.c_double
+    lib.oracle_attn_f64.argtypes = [dp, dp, dp, dp, dp, c_int, c_int, c_int,
+                                    c_int, c_double, c_int, i32p, c_int]
+    lib.oracle_attn_f64.restype = c_int
+    lib.oracle_attn_bf16.argtypes = [u16p, u16p, u16p, dp, dp, c_int, c_int,
+                                     c_int, c_int, c_double, c_int, i32p, i32p,
+                                     c_int, c_int]
+    lib.oracle_attn_bf16.restype = c_int
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = c_int
+    return lib
+
+
+def load(path: str = _LIB_PATH):
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    if path != _LIB_PATH:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            if (not os.path.exists(_LIB_PATH)
+                    or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+                build()
+            _lib = _bind(ctypes.CDLL(_LIB_PATH))
+        return _lib
+
+
+def max_threads() -> int:
+    return int(load().oracle_max_threads())
+
+
+def _as_numpy(x):
+    """torch tensor or array -> (numpy array, is_bf16)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return x.view(torch.int16).numpy().view(np.uint16), True
+            return x.to(torch.float64).numpy(), False
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(x)
+    if a.dtype == np.uint16:
+        return a, True
+    return np.ascontiguousarray(a, dtype=np.float64), False
+
+
+def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
+              nthreads=0, lib=None):
+    """Exact attention in fp64.
+
+    q, k, v: [B, H, N, d] as torch bf16 / float tensors or numpy arrays
+    (uint16 arrays are read as bf16 bit patterns). kv_len: None or [B] ints.
+    rows: None (all rows) or a list of query-row indices evaluated in every
+    (b, h). Returns (o [B,H,R,d] float64, lse [B,H,R] float64), R = N or
+    len(rows).
+    """
+    lib = lib or load()
+    qa, qb16 = _as_numpy(q)
+    ka, kb16 = _as_numpy(k)
+    va, vb16 = _as_numpy(v)
+    if not (qb16 == kb16 == vb16):
+        raise TypeError("q, k, v must share one element type")
+    if qa.ndim != 4 or qa.shape != ka.shape or qa.shape != va.shape:
+        raise ValueError(f"bad shapes {qa.shape} {ka.shape} {va.shape}")
+    B, H, N, d = qa.shape
+    kvp = None
+    if kv_len is not None:
+        kvl = np.ascontiguousarray(np.asarray(
+            kv_len.cpu().numpy() if hasattr(kv_len, "cpu") else kv_len,
+            dtype=np.int32))
+        if kvl.shape != (B,):
+            raise ValueError("kv_len must have shape [B]")
+        kvp = kvl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    R = N if rows is None else len(rows)
+    o = np.zeros((B, H, R, d), dtype=np.float64)
+    lse = np.zeros((B, H, R), dtype=np.float64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    if qb16:
+        rp = None
+        if rows is not None:
+            ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+            rp = ra.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        rc = lib.oracle_attn_bf16(qa.ctypes.data_as(u16p), ka.ctypes.data_as(u16p),
+                                  va.ctypes.data_as(u16p), o.ctypes.data_as(dp),
+                                  lse.ctypes.data_as(dp), B, H, N, d, float(scale),
+                                  int(bool(causal)), kvp, rp, R, int(nthreads))
+    else:
+        if rows is not None:
+            raise ValueError("row subsets are supported for bf16 inputs only")
+        rc = lib.oracle_attn_f64(qa.ctypes.data_as(dp), ka.ctypes.data_as(dp),
+                                 va.ctypes.data_as(dp), o.ctypes.data_as(dp),
+                                 lse.ctypes.data_as(dp), B, H, N, d, float(scale),
+                                 int(bool(causal)), kvp, int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle returned error {rc}")
+    return o, lse

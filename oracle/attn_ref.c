@@ -1,0 +1,221 @@
+/*
+ * CPU oracle for exact attention: TEST INFRASTRUCTURE ONLY.
+ *
+ * Only the test suite, the smoke check and the benchmark's CPU-baseline /
+ * reference leg load this library. The product path (the CUDA library) never
+ * calls it, links it or shares code with it.
+ *
+ * What it computes is the plain definition of scaled dot-product attention as
+ * the FlashAttention pages state it ("FlashAttention (UR)", section "Problem
+ * of standard attention": Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V),
+ * with the mask added to the scores before the softmax (the fused operation
+ * chain in section "Fusing operations into one CUDA kernel" lists masking
+ * between Q K^T and the softmax). It is the "standard" implementation those
+ * pages contrast with the fused one: every score of a query row is
+ * materialised, then the softmax is taken in two passes (max, then sum of
+ * exponentials) over the whole row. No tiling, no online rescaling.
+ *
+ * Readings taken where the pages are silent:
+ *   - scale is passed by the caller (1/sqrt(d) in every workload);
+ *   - the mask is additive -inf; causal means key j is allowed iff j <= i
+ *     (square, N_q == N_k); key padding masks keys j >= kv_len[b], and query
+ *     rows beyond kv_len[b] are still computed against the valid keys;
+ *   - a row with no allowed key gets O = 0 and lse = -inf;
+ *   - lse_i = ln sum_j exp(s_ij), natural log, scale included.
+ *
+ * Arithmetic: IEEE fp64 throughout. bf16 inputs are widened exactly (a bf16
+ * value is the top 16 bits of an fp32, and fp32 -> fp64 is exact).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL 1
+#define ORACLE_ENOMEM 2
+
+static double bf16_to_f64(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Is key j visible to query row i? */
+static int key_allowed(int i, int j, int causal, int kv_lim)
+{
+    if (j >= kv_lim) return 0;
+    if (causal && j > i) return 0;
+    return 1;
+}
+
+/*
+ * One query row against one head's K and V (row-major [N][d] fp64).
+ * srow is caller scratch of N doubles: the materialised score row.
+ */
+static void attn_one_row(const double *qi, const double *K, const double *V,
+                         int N, int d, double scale, int i, int causal,
+                         int kv_lim, double *srow, double *oi, double *lse_i)
+{
+    /* s_ij = scale * <q_i, k_j> + mask_ij */
+    for (int j = 0; j < N; ++j) {
+        if (!key_allowed(i, j, causal, kv_lim)) {
+            srow[j] = -INFINITY;
+            continue;
+        }
+        const double *kj = K + (size_t)j * d;
+        double dot = 0.0;
+        for (int t = 0; t < d; ++t) dot += qi[t] * kj[t];
+        srow[j] = scale * dot;
+    }
+    /* pass 1: row max */
+    double m = -INFINITY;
+    for (int j = 0; j < N; ++j)
+        if (srow[j] > m) m = srow[j];
+    for (int t = 0; t < d; ++t) oi[t] = 0.0;
+    if (m == -INFINITY) { /* no visible key */
+        *lse_i = -INFINITY;
+        return;
+    }
+    /* pass 2: sum of exponentials, then the normaliser */
+    double sum = 0.0;
+    for (int j = 0; j < N; ++j)
+        if (srow[j] != -INFINITY) sum += exp(srow[j] - m);
+    double lse = m + log(sum);
+    /* O_i = sum_j softmax_ij * v_j */
+    for (int j = 0; j < N; ++j) {
+        if (srow[j] == -INFINITY) continue;
+        double p = exp(srow[j] - lse);
+        const double *vj = V + (size_t)j * d;
+        for (int t = 0; t < d; ++t) oi[t] += p * vj[t];
+    }
+    *lse_i = lse;
+}
+
+static int check_args(int B, int H, int N, int d, double scale, int causal)
+{
+    if (B < 0 || H < 0 || N < 0 || d <= 0) return ORACLE_EINVAL;
+    if (!(scale == scale) || isinf(scale)) return ORACLE_EINVAL;
+    if (causal != 0 && causal != 1) return ORACLE_EINVAL;
+    return ORACLE_OK;
+}
+
+/*
+ * Shared driver. Inputs are either fp64 (qd/kd/vd) or bf16 bit patterns
+ * (qb/kb/vb); exactly one set is non-null. `rows` (nullable) selects which
+ * query rows of every head to compute; outputs are then [B,H,nrows,d] and
+ * [B,H,nrows]. With rows == NULL, nrows must equal N and all rows are done.
+ */
+static int attn_driver(const double *qd, const double *kd, const double *vd,
+                       const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
+                       double *o, double *lse, int B, int H, int N, int d,
+                       double scale, int causal, const int32_t *kv_len,
+                       const int32_t *rows, int nrows, int nthreads)
+{
+    int rc = check_args(B, H, N, d, scale, causal);
+    if (rc) return rc;
+    if (nrows < 0 || (rows == NULL && nrows != N)) return ORACLE_EINVAL;
+    if (rows)
+        for (int r = 0; r < nrows; ++r)
+            if (rows[r] < 0 || rows[r] >= N) return ORACLE_EINVAL;
+    if (B == 0 || H == 0 || nrows == 0) return ORACLE_OK;
+    if (N == 0) return ORACLE_EINVAL; /* rows must index into N */
+
+    const size_t head = (size_t)N * d;
+    const int widen = (qb != NULL);
+    double *Kh = NULL, *Vh = NULL, *Qh = NULL;
+    if (widen) {
+        Kh = (double *)malloc(head * sizeof(double));
+        Vh = (double *)malloc(head * sizeof(double));
+        Qh = (double *)malloc(head * sizeof(double));
+        if (!Kh || !Vh || !Qh) {
+            free(Kh); free(Vh); free(Qh);
+            return ORACLE_ENOMEM;
+        }
+    }
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int err = ORACLE_OK;
+    for (int b = 0; b < B; ++b) {
+        int kv_lim = N;
+        if (kv_len) {
+            kv_lim = kv_len[b];
+            if (kv_lim < 0) kv_lim = 0;
+            if (kv_lim > N) kv_lim = N;
+        }
+        for (int h = 0; h < H; ++h) {
+            const size_t base = ((size_t)b * H + h) * head;
+            const double *Q, *K, *V;
+            if (widen) {
+                for (size_t e = 0; e < head; ++e) {
+                    Qh[e] = bf16_to_f64(qb[base + e]);
+                    Kh[e] = bf16_to_f64(kb[base + e]);
+                    Vh[e] = bf16_to_f64(vb[base + e]);
+                }
+                Q = Qh; K = Kh; V = Vh;
+            } else {
+                Q = qd + base; K = kd + base; V = vd + base;
+            }
+            double *o_bh = o + ((size_t)b * H + h) * (size_t)nrows * d;
+            double *l_bh = lse + ((size_t)b * H + h) * (size_t)nrows;
+#pragma omp parallel
+            {
+                double *srow = (double *)malloc((size_t)N * sizeof(double));
+                if (!srow) {
+#pragma omp atomic write
+                    err = ORACLE_ENOMEM;
+                } else {
+#pragma omp for schedule(dynamic, 4)
+                    for (int r = 0; r < nrows; ++r) {
+                        int i = rows ? rows[r] : r;
+                        attn_one_row(Q + (size_t)i * d, K, V, N, d, scale, i,
+                                     causal, kv_lim, srow,
+                                     o_bh + (size_t)r * d, l_bh + r);
+                    }
+                    free(srow);
+                }
+            }
+        }
+    }
+    free(Kh); free(Vh); free(Qh);
+    return err;
+}
+
+/* fp64 inputs, all rows. q,k,v: [B,H,N,d]; o: [B,H,N,d]; lse: [B,H,N]. */
+int oracle_attn_f64(const double *q, const double *k, const double *v,
+                    double *o, double *lse, int B, int H, int N, int d,
+                    double scale, int causal, const int32_t *kv_len,
+                    int nthreads)
+{
+    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
+    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, N, d, scale,
+                       causal, kv_len, NULL, N, nthreads);
+}
+
+/* bf16 bit-pattern inputs; optional row subset (rows may be NULL => nrows == N). */
+int oracle_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     double *o, double *lse, int B, int H, int N, int d,
+                     double scale, int causal, const int32_t *kv_len,
+                     const int32_t *rows, int nrows, int nthreads)
+{
+    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
+    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, N, d, scale,
+                       causal, kv_len, rows, nrows, nthreads);
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

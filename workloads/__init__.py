@@ -1,0 +1,124 @@
+"""Seeded synthetic attention workloads.
+
+This module only draws random numbers and describes shapes. It holds none of
+the attention arithmetic, so that the CPU oracle and the CUDA path can both be
+fed from it without sharing any of the method's code.
+
+The five workloads take the shapes of the experiments the FlashAttention pages
+report ("FlashAttention (UR)", section "Experimental results": BERT-large at
+length 512, GPT-2 at length 1K, Long-Range Arena at 1K-4K) plus a tiny
+correctness case and a long-context single-batch case. No model, weights or
+dataset is involved: every tensor is i.i.d. N(0, 1) rounded to bfloat16.
+
+Recipe (fixed, so any run can be reproduced):
+  * generator: ``torch.Generator('cpu').manual_seed(seed)``;
+  * draw order: Q, then K, then V, each ``torch.randn([B, H, N, d])`` in fp32,
+    then ``.to(torch.bfloat16)`` (round to nearest even);
+  * ``q_mult`` (long-range case): Q is multiplied by 4 after rounding, which is
+    exact in bf16 because 4 is a power of two;
+  * key padding (BERT-shaped case): after V,
+    ``kv_len = torch.randint(kv_lo, kv_hi + 1, (B,))`` from the same generator;
+  * default seed: the workload's index (1..5).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    index: int
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    q_mult: float = 1.0
+    kv_len_range: Optional[tuple] = None  # (lo, hi) inclusive, or None
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def units(self) -> int:
+        """Query tiles of 128 rows: the independent work units."""
+        return self.B * self.H * ((self.N + 127) // 128)
+
+    def flops(self) -> float:
+        """Counted FLOPs of the metric: 4*B*H*N^2*d, halved when causal."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def describe(self) -> dict:
+        return {
+            "workload": self.name,
+            "B": self.B, "H": self.H, "N": self.N, "d": self.d,
+            "causal": self.causal,
+            "mask": ("causal" if self.causal else
+                     ("key_padding" if self.kv_len_range else "none")),
+            "q_mult": self.q_mult,
+            "scale": self.scale,
+        }
+
+
+WORKLOADS = [
+    Workload("tiny_noncausal_B1_H2_N256_d64", 1, 1, 2, 256, 64, False),
+    Workload("bert_large_keypad_B16_H16_N512_d64", 2, 16, 16, 512, 64, False,
+             kv_len_range=(256, 512)),
+    Workload("gpt2_causal_B8_H12_N1024_d64", 3, 8, 12, 1024, 64, True),
+    Workload("long_range_causal_qx4_B2_H16_N4096_d128", 4, 2, 16, 4096, 128, True,
+             q_mult=4.0),
+    Workload("long_context_causal_B1_H32_N16384_d128", 5, 1, 32, 16384, 128, True),
+]
+
+BY_NAME = {w.name: w for w in WORKLOADS}
+BY_INDEX = {w.index: w for w in WORKLOADS}
+
+
+def get(key) -> Workload:
+    if isinstance(key, int):
+        return BY_INDEX[key]
+    if isinstance(key, str) and key.isdigit():
+        return BY_INDEX[int(key)]
+    return BY_NAME[key]
+
+
+def make_inputs(w: Workload, seed: Optional[int] = None):
+    """Return (q, k, v, kv_len) on the CPU; q/k/v bf16 [B,H,N,d], kv_len int32 [B] or None."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.index if seed is None else seed)
+    shape = (w.B, w.H, w.N, w.d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    if w.q_mult != 1.0:
+        q = q * w.q_mult
+    kv_len = None
+    if w.kv_len_range is not None:
+        lo, hi = w.kv_len_range
+        kv_len = torch.randint(lo, hi + 1, (w.B,), generator=g).to(torch.int32)
+    return q, k, v, kv_len
+
+
+def make_custom(B, H, N, d, seed, q_mult=1.0, kv_len_range=None):
+    """Same recipe for an arbitrary shape (ragged-tail and edge-case tests)."""
+    w = Workload(f"custom_B{B}_H{H}_N{N}_d{d}", 0, B, H, N, d, False, q_mult,
+                 kv_len_range)
+    return make_inputs(w, seed=seed)
+
+
+def sample_rows(N: int, seed: int, n_random: int = 256, edge: int = 128):
+    """Row indices for sampled checks at full size: the first and last `edge`
+    rows plus `n_random` seeded random rows, sorted and unique."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    rows = set(range(min(edge, N))) | set(range(max(0, N - edge), N))
+    if N > 0:
+        rows |= set(torch.randint(0, N, (n_random,), generator=g).tolist())
+    return sorted(rows)
