@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 5]
+
+A step is one full forward (one kernel launch) over the workload's tensors,
+which are resident in device memory before the timed region starts. The
+default workload is the long-context causal case (B=1, H=32, N=16384, d=128),
+the largest configuration; its inputs (3 x 128 MiB) exceed the 126 MB L2, so
+no L2 flush is done between steps. Metric: counted FLOPs 4*B*H*N^2*d (half
+when causal) per second, in TFLOP/s.
+
+With N > 1 GPUs (torchrun, one process per GPU) every rank runs its own
+replica of the workload (own seed): there is no data exchange on the path,
+only a barrier and a max-reduction of the timings ("scaling": "weak").
+
+--impl reference times the CPU oracle (fp64 C, the machine's host cores) on a
+bounded row sample of the same workload, in the same unit; under torchrun only
+rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = ("attention fwd TFLOP/s (4·B·H·N²·d) and % of B200 "
+          "dense BF16 peak")
+UNIT = "TFLOP/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["io_aware_exact_18_b200/csrc/fa_fwd_kernel.cuh",
+                  "io_aware_exact_18_b200/csrc/sm100_ptx.cuh",
+                  "io_aware_exact_18_b200/csrc/fa_api.cu"]
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; otherwise None."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line:
+                key, val = line.split(":", 1)
+                vals[key.strip()] = val.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling in the background (200 ms period)."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self._proc = None
+        self._thread = None
+
+    def start(self):
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self._proc = None
+            return
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+
+    def _read(self):
+        for line in self._proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1]
+        window = "timed"
+        if len(inside) < 3:
+            inside = [p for (_, p) in self.samples]
+            window = "warmup+timed"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = sorted(v for v in (num(p[1]) for p in inside) if v is not None)
+        smax = max((v for v in (num(p[2]) for p in inside) if v is not None), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4)
+                          if p[5 + i].lower() == "active"})
+        pw = [v for v in (num(p[3]) for p in inside) if v is not None]
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(inside), "window": window,
+                "power_w_max": max(pw) if pw else None}
+
+
+# ----------------------------------------------------------------- CPU oracle sample
+def oracle_sample_rows(w, budget_s, seed, nthreads, q, k, v, kv_len, max_rows=None):
+    """Time the oracle on a seeded row sample sized to about `budget_s`.
+
+    Returns (seconds, counted_flops, description). Counted FLOPs of a row are
+    4*d*(visible keys of that row); summed over all rows this is the
+    metric's count."""
+    import numpy as np
+    import oracle
+    N, d = w.N, w.d
+    rng = np.random.default_rng(seed)
+
+    def visible(i, b):
+        lim = N
+        if kv_len is not None:
+            lim = int(min(max(int(kv_len[b]), 0), N))
+        return min(lim, i + 1) if w.causal else lim
+
+    def run(rows):
+        t = time.perf_counter()
+        oracle.attention(q, k, v, w.scale, causal=w.causal, kv_len=kv_len, rows=rows,
+                         nthreads=nthreads)
+        dt = time.perf_counter() - t
+        fl = sum(4.0 * d * visible(i, b) for b in range(w.B) for i in rows) * w.H
+        return dt, fl
+
+    probe = sorted(set(rng.integers(0, N, size=4).tolist()))
+    dt, fl = run(probe)
+    rate = fl / max(dt, 1e-6)
+    avg_row_flops = fl / max(len(probe), 1)
+    n_rows = int(max(4, min(N, budget_s * rate / max(avg_row_flops, 1.0))))
+    if max_rows is not None:
+        n_rows = min(n_rows, max_rows)
+    rows = sorted(set(rng.integers(0, N, size=n_rows).tolist()))
+    dt, fl = run(rows)
+    desc = (f"{len(rows)} seeded random query rows x all {w.B * w.H} (b,h) heads of "
+            f"{w.name} (fraction {len(rows) / N:.4f} of the rows), fp64, "
+            f"{nthreads} threads")
+    return dt, fl, desc
+
+
+def reference_arm(args, w):
+    """CPU oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    q, k, v, kv_len = workloads.make_inputs(w)
+    nthreads = os.cpu_count() or 1
+    oracle.load()
+    per_step = max(0.2, min(5.0, 150.0 / max(args.steps + args.warmup, 1)))
+    for i in range(args.warmup):
+        oracle_sample_rows(w, per_step / 4, 10 + i, nthreads, q, k, v, kv_len)
+    tot_t, tot_f, desc = 0.0, 0.0, ""
+    for i in range(args.steps):
+        dt, fl, desc = oracle_sample_rows(w, per_step, 1000 + i, nthreads, q, k, v, kv_len)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    # ms per step expressed for the whole workload (extrapolated from the samples)
+    ms_full = w.flops() / (value * 1e12) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_full, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**w.describe(), "l2": "n/a (CPU)",
+                   "note": "per-step time extrapolated from the row sample"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() \
+        and dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def our_arm(args, w):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import io_aware_exact_18_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.load_library()
+
+    # ---- inputs resident in HBM before the timed region
+    q, k, v, kv_len = workloads.make_inputs(w, seed=w.index + 1000 * rank)
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    kvd = None if kv_len is None else kv_len.to(dev)
+    od = torch.empty_like(qd)
+    lsed = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+
+    def step():
+        if kvd is None:
+            st = fa.fa_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                           lsed.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal), sh)
+        else:
+            st = fa.fa_fwd_kvlen(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                                 lsed.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal),
+                                 kvd.data_ptr(), sh)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_fwd")
+
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    sampler.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    st = fa.fa_last_device_error(sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "warm-up")
+
+    # ---- timed region: device events on the launching stream
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    st = fa.fa_last_device_error(sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed region")
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    flops = w.flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.steps, 10))
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    kvh = None if kv_len is None else kv_len.pin_memory()
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    lh = torch.empty(lsed.shape, dtype=lsed.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh)) + \
+        (0 if kvh is None else kvh.numel() * kvh.element_size())
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            if kvh is not None:
+                kvd.copy_(kvh, non_blocking=True)
+            fa.attention(qd, kd, vd, scale=w.scale, causal=w.causal, kv_len=kvd, out=od,
+                         lse=lsed, stream=sh)
+            oh.copy_(od, non_blocking=True)
+            lh.copy_(lsed, non_blocking=True)
+
+    e2e_step()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    st = fa.fa_last_device_error(sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "e2e")
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    # ---- roofline of the (only) kernel: one launch per step
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_local * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = recorded_traffic(w.name)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+                "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
+                "algorithmic_bytes": float(w.B * w.H * w.N * (4 * w.d * 2 + 4)),
+                "kernel": f"fa_fwd_sm100<{w.d}>"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nthreads = os.cpu_count() or 1
+        dt, fl, desc = oracle_sample_rows(w, args.cpu_seconds, 7, nthreads, q, k, v, kv_len)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+               "sample": desc, "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {**w.describe(), "parallelism": f"replicas x{world}",
+                       "l2": "no flush: inputs (3 x {:.0f} MiB) exceed the 126 MB L2".format(
+                           w.B * w.H * w.N * w.d * 2 / 2**20)},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="5", help="workload index (1-5) or name")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    w = workloads.get(args.workload)
+    if args.impl == "reference":
+        return reference_arm(args, w)
+    return our_arm(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

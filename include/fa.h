@@ -1,0 +1,95 @@
+/*
+ * fa.h -- C ABI of the exact, fused attention forward library (libfa.so).
+ *
+ * The operation is the attention of "FlashAttention (UR)", section "Problem
+ * of standard attention":
+ *
+ *     O = softmax(scale * Q K^T + mask) V,      lse_i = ln sum_j exp(s_ij)
+ *
+ * with s_ij = scale * <q_i, k_j> + mask_ij and mask_ij = -inf for hidden keys
+ * (masking sits between Q K^T and the softmax in the fused chain of section
+ * "Fusing operations into one CUDA kernel"). It is evaluated tile by tile
+ * with an online softmax (section "Online softmax") so the N x N score matrix
+ * never reaches device memory, and the per-row log-sum-exp is emitted as the
+ * O(N) statistic (section "Complexity and optimality").
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller. The library allocates
+ *     no device memory per call and keeps no reference after it returns.
+ *   - Layout: q, k, v, o are bf16 [B, H, N, d], contiguous, d innermost
+ *     (row (b,h,i) starts at element ((b*H + h)*N + i)*d). lse is fp32
+ *     [B, H, N], natural log, scale included.
+ *   - q, k, v, o must be 16-byte aligned (the tensor-memory-access engine
+ *     requires it); lse 4-byte aligned. o and lse must not overlap each other
+ *     or the inputs.
+ *   - d must be 64 or 128; anything else returns FA_ERR_UNSUPPORTED.
+ *   - B, H, N >= 0. If any is 0 there is nothing to compute: the call returns
+ *     FA_OK without launching (pointers may then be NULL).
+ *   - scale must be finite and > 0; causal must be 0 or 1.
+ *   - Causal masking is square: query row i sees key j iff j <= i.
+ *   - A row with no visible key gets O = 0 and lse = -inf.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls are
+ *     asynchronous: they return once the kernel is enqueued. q, k, v are only
+ *     read; every element of o and lse is written.
+ *   - Argument errors are reported synchronously and launch nothing.
+ *   - Results are deterministic: identical inputs give bitwise identical
+ *     outputs on the same GPU (the method is exact and deterministic,
+ *     "FlashAttention-2 (HI)", section "Performance and efficiency").
+ *   - Requires a B200-class GPU (compute capability 10.0, sm_100a); other
+ *     devices get FA_ERR_UNSUPPORTED. There is no CPU fallback.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null/misaligned/overlapping pointer, bad size, scale, causal */
+    FA_ERR_UNSUPPORTED = 2,  /* head dim other than 64/128, or not an sm_100 device */
+    FA_ERR_LAUNCH = 3,       /* the CUDA runtime refused the launch or a sync failed */
+    FA_ERR_TIMEOUT = 4       /* a kernel's bounded wait ran out (see fa_last_device_error) */
+} fa_status_t;
+
+/*
+ * Exact attention forward, optional causal mask.
+ * q, k, v: bf16 [B,H,N,d] in; o: bf16 [B,H,N,d] out; lse: fp32 [B,H,N] out.
+ * Returns an fa_status_t value.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int H, int N, int d, float scale, int causal, void *stream);
+
+/*
+ * Same, plus a per-sequence key-padding mask: keys j >= kv_len[b] are hidden
+ * from every query row of batch b (query rows past kv_len[b] are still
+ * computed against the visible keys). kv_len: device int32 [B], or NULL for
+ * "all N keys visible". Values are clamped to [0, N]; 0 hides every key.
+ * The pages name masking inside the fused kernel but no mask interface; a
+ * valid length per sequence is the plainest form that keeps an N x N mask
+ * out of device memory.
+ */
+int fa_fwd_kvlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                 int B, int H, int N, int d, float scale, int causal,
+                 const int32_t *kv_len, void *stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word, which kernels set when a bounded wait runs out (FA_ERR_TIMEOUT). The
+ * word is sticky: while it is set, later launches on that device skip their
+ * work, so call this after any call whose results matter. Returns FA_OK,
+ * FA_ERR_TIMEOUT, or FA_ERR_LAUNCH if the synchronisation itself failed.
+ */
+int fa_last_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,130 @@
+"""Exact, IO-aware fused attention forward for B200 (sm_100a).
+
+Thin ctypes binding over ``libfa.so`` (C ABI declared in ``include/fa.h``).
+Every function here only marshals arguments; all arithmetic runs in the CUDA
+kernels of the library. There is no CPU fallback: if the library is missing
+or the device is not an sm_100 GPU, calls fail loudly.
+
+Names follow the C ABI: :func:`fa_fwd`, :func:`fa_fwd_kvlen`,
+:func:`fa_status_string`, :func:`fa_last_device_error`. :func:`attention` is
+a convenience wrapper that allocates the outputs with torch and calls
+:func:`fa_fwd` / :func:`fa_fwd_kvlen` on the current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fa.h")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_LAUNCH = 3
+FA_ERR_TIMEOUT = 4
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}{': ' if what else ''}{fa_status_string(status)} ({status})")
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libfa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(
+            f"CUDA extension missing: {path} (build it with "
+            "`python -m io_aware_exact_18_b200.build`)")
+    lib = ctypes.CDLL(path)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_fwd_kvlen.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
+    lib.fa_fwd_kvlen.restype = i
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_device_error.argtypes = [vp]
+    lib.fa_last_device_error.restype = i
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def declared_symbols(header: str = HEADER_PATH):
+    """Function names declared in include/fa.h."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream) -> int:
+    """C ABI fa_fwd; q,k,v,o,lse and stream are raw integers (device pointers, cudaStream_t)."""
+    return load_library().fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream)
+
+
+def fa_fwd_kvlen(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, stream) -> int:
+    """C ABI fa_fwd_kvlen; kv_len is a device pointer to int32 [B] or 0/None."""
+    return load_library().fa_fwd_kvlen(q, k, v, o, lse, B, H, N, d, scale, causal,
+                                       kv_len, stream)
+
+
+def fa_status_string(status: int) -> str:
+    try:
+        return load_library().fa_status_string(int(status)).decode()
+    except ImportError:
+        return f"status {status}"
+
+
+def fa_last_device_error(stream) -> int:
+    return load_library().fa_last_device_error(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def attention(q, k, v, scale=None, causal=False, kv_len=None, out=None, lse=None,
+              stream=None, check=True):
+    """O, lse = attention(q, k, v) for bf16 CUDA tensors [B, H, N, d].
+
+    Allocates O (bf16) and lse (fp32) unless given, calls the C ABI on the
+    current torch stream (or `stream`), and raises FAError on a bad status.
+    """
+    import torch
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("q, k, v must be bfloat16")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors (no CPU fallback)")
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError(f"q, k, v must share one [B,H,N,d] shape, got {q.shape} {k.shape} {v.shape}")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device).cuda_stream
+    if kv_len is None:
+        st = fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
+                    float(scale), int(bool(causal)), s)
+    else:
+        if kv_len.dtype != torch.int32 or not kv_len.is_cuda or kv_len.shape != (B,):
+            raise ValueError("kv_len must be a CUDA int32 tensor of shape [B]")
+        st = fa_fwd_kvlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
+                          float(scale), int(bool(causal)), _ptr(kv_len), s)
+    if check and st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return out, lse

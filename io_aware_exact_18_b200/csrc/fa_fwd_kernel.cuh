@@ -1,0 +1,419 @@
+// Fused exact attention forward for sm_100a (B200).
+//
+// Computes O = softmax(scale * Q K^T + mask) V and lse = ln sum_j exp(s_ij)
+// for bf16 Q, K, V laid out [B, H, N, d] (d innermost), accumulating in fp32.
+// The N x N score matrix never leaves the SM: each 128 x 128 score tile lives
+// in tensor memory (TMEM), is turned into probabilities there, and feeds the
+// P.V product directly ("FlashAttention (UR)", sections "Tiling and block
+// processing" and "Fusing operations into one CUDA kernel").
+//
+// Softmax is evaluated online, one key tile at a time, with a running row
+// maximum m and running sum of exponentials l ("FlashAttention (UR)", section
+// "Online softmax"). Exponentials use base 2 with the scale folded into one
+// FFMA per score, and the division by l is deferred to the epilogue, which
+// trims the non-matmul work that "FlashAttention-2 (HI)" section 1 targets.
+// The O accumulator is rescaled only when a row maximum grows by more than
+// 2^8 (in the log2 domain); otherwise the stale maximum keeps being used as
+// the reference. Both O and l share that reference, so the final O / l is
+// unchanged by this choice (the ratio is exact), and probabilities stay below
+// 2^8, far from fp32 or bf16 overflow.
+//
+// Work partitioning ("FlashAttention-2 (HI)", sections 2 and 3): the grid is
+// batch x heads x (pairs of 128-row query tiles), so one long head still fills
+// every SM; the heaviest causal tiles are launched first. Inside a CTA the
+// work is split by role rather than by rows of the same tile:
+//   warps 0-3   softmax for query tile 0 (thread r owns row r = TMEM lane r)
+//   warps 4-7   softmax for query tile 1
+//   warp  8     issues tcgen05 MMAs (one thread) and owns the TMEM allocation
+//   warp  9     issues TMA loads (one thread)
+// With one thread per row no cross-thread reduction is needed for the row
+// max and row sum. The two softmax warpgroups ping-pong: while one works on
+// its score tile the tensor cores run the other tile's P.V and next Q.K^T.
+//
+// TMEM (512 columns x 128 lanes of 32 bit):
+//   [0,128)    S0 (fp32 scores of tile 0); P0 (bf16 pairs) overwrites [0,64)
+//   [128,256)  S1 / P1
+//   [256,256+d)      O0 accumulator (fp32)
+//   [256+d,256+2d)   O1 accumulator
+// Shared memory: Q0, Q1 and a ring of K/V slots, each a 128-row tile stored
+// as d/64 column blocks of 128 rows x 128 bytes in the 128-byte swizzled
+// layout that TMA writes and tcgen05 descriptors read.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+constexpr int kTile = 128;         // rows per query tile and keys per KV tile
+constexpr int kThreads = 320;      // 2 softmax warpgroups + MMA warp + TMA warp
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D>
+struct Cfg {
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static constexpr int kBlocks = D / 64;                // 128-byte column blocks per row
+    static constexpr int kBlockBytes = kTile * 128;       // 16 KB
+    static constexpr int kTileBytes = kTile * D * 2;      // one Q/K/V tile
+    static constexpr int kSlots = (D == 128) ? 4 : 8;     // K/V ring depth
+    static constexpr int kSmemTiles = (2 + kSlots) * kTileBytes;
+    static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 512 /*barriers*/;
+    static constexpr uint32_t kTmemCols = 512;
+    __device__ static constexpr uint32_t col_s(int t) { return (uint32_t)(t * 128); }
+    __device__ static constexpr uint32_t col_o(int t) { return 256u + (uint32_t)(t * D); }
+};
+
+struct FwdParams {
+    __nv_bfloat16* o;          // [B,H,N,d]
+    float* lse;                // [B,H,N]
+    const int32_t* kv_len;     // [B] or nullptr
+    uint32_t* dev_err;         // status word
+    int B, H, N;
+    int n_pairs;               // ceil(N / 256)
+    int causal;
+    float scale_log2;          // scale * log2(e)
+    uint64_t watchdog_ns;
+};
+
+struct SmemBarriers {
+    uint64_t q_full[2];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_done[2];
+    uint64_t teardown;
+    uint64_t kv_full[8];
+    uint64_t kv_empty[8];
+    uint32_t tmem_base;
+    int abort;
+    int skip;
+};
+
+// Number of 128-key tiles query tile `t` of this CTA must visit.
+__device__ __forceinline__ int kv_tiles_for(int q_first, int N, int kv_lim, int causal) {
+    if (q_first >= N) return 0;
+    int lim = kv_lim;
+    if (causal) lim = min(lim, q_first + kTile);
+    return (lim + kTile - 1) / kTile;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using C = Cfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ[2] = {smem, smem + C::kTileBytes};
+    uint8_t* sKV = smem + 2 * C::kTileBytes;
+    SmemBarriers* bars = reinterpret_cast<SmemBarriers*>(smem + C::kSmemTiles);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // ---------------------------------------------------------- work unit
+    // Head-major order keeps one head's K/V resident in L2 while its query
+    // tiles run; within a head the heaviest (last, for causal) pair goes first.
+    const int bh = (int)(blockIdx.x / (unsigned)p.n_pairs);
+    const int pair = p.n_pairs - 1 - (int)(blockIdx.x % (unsigned)p.n_pairs);
+    const int b = bh / p.H;
+    const int q0 = pair * 2 * kTile;
+    int kv_lim = p.N;
+    if (p.kv_len != nullptr) kv_lim = max(0, min(p.N, p.kv_len[b]));
+    int n_t[2];
+    n_t[0] = kv_tiles_for(q0, p.N, kv_lim, p.causal);
+    n_t[1] = kv_tiles_for(q0 + kTile, p.N, kv_lim, p.causal);
+    const int n_max = max(n_t[0], n_t[1]);
+
+    // ---------------------------------------------------------- setup
+    if (tid == 0) {
+        mbar_init(&bars->q_full[0], 1);
+        mbar_init(&bars->q_full[1], 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars->s_full[t], 1);
+            mbar_init(&bars->p_full[t], kTile);
+            mbar_init(&bars->o_done[t], 1);
+        }
+        mbar_init(&bars->teardown, 1);
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(&bars->kv_full[s], 1);
+            mbar_init(&bars->kv_empty[s], 1);
+        }
+        bars->abort = 0;
+        bars->skip = (*reinterpret_cast<volatile uint32_t*>(p.dev_err) != 0u) ? 1 : 0;
+        fence_mbarrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&bars->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const bool skip = bars->skip != 0;
+    const Watchdog wd{&bars->abort, p.dev_err, p.watchdog_ns};
+
+    if (warp == kTmaWarp) {
+        // ====================================================== TMA producer
+        if (lane == 0 && !skip) {
+            const uint64_t pol_kv = policy_evict_last();
+            const uint64_t pol_q = policy_evict_first();
+            for (int t = 0; t < 2; ++t) {
+                if (n_t[t] == 0) continue;
+                mbar_arrive_expect_tx(&bars->q_full[t], C::kTileBytes);
+                for (int blk = 0; blk < C::kBlocks; ++blk)
+                    tma_load_3d_hint(&tm_q, &bars->q_full[t], sQ[t] + blk * C::kBlockBytes,
+                                     blk * 64, q0 + t * kTile, bh, pol_q);
+            }
+            int issued = 0;
+            for (int L = 0; L < 2 * n_max; ++L) {
+                const int slot = L % C::kSlots;
+                const uint32_t round = (uint32_t)(L / C::kSlots);
+                if (!mbar_wait(&bars->kv_empty[slot], (round & 1u) ^ 1u, wd)) break;
+                const CUtensorMap* map = (L & 1) ? &tm_v : &tm_k;
+                uint8_t* dst = sKV + slot * C::kTileBytes;
+                mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
+                for (int blk = 0; blk < C::kBlocks; ++blk)
+                    tma_load_3d_hint(map, &bars->kv_full[slot], dst + blk * C::kBlockBytes,
+                                     blk * 64, (L >> 1) * kTile, bh, pol_kv);
+                issued = L + 1;
+            }
+            // Drain: every load issued must have landed before the CTA exits.
+            for (int L = max(0, issued - C::kSlots); L < issued; ++L)
+                mbar_wait_drain(&bars->kv_full[L % C::kSlots], (uint32_t)(L / C::kSlots) & 1u,
+                                wd);
+            for (int t = 0; t < 2; ++t)
+                if (n_t[t] > 0) mbar_wait_drain(&bars->q_full[t], 0u, wd);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ====================================================== MMA issuer
+        if (lane == 0 && !skip) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTile, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+            auto issue_qk = [&](int t, int slot) {
+                const uint32_t a0 = smem_u32(sQ[t]);
+                const uint32_t b0 = smem_u32(sKV + slot * C::kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * C::kBlockBytes + (kk & 3) * 32);
+                    umma_ss(tmem + C::col_s(t), smem_desc_sw128(a0 + off, 16, 1024),
+                            smem_desc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int t, int slot, bool accumulate) {
+                const uint32_t b0 = smem_u32(sKV + slot * C::kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + (uint32_t)(kk * 8),
+                            smem_desc_sw128(b0 + (uint32_t)(kk * 16 * 128), C::kBlockBytes, 1024),
+                            idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = true;
+            for (int t = 0; t < 2 && ok; ++t)
+                if (n_t[t] > 0) ok = mbar_wait(&bars->q_full[t], 0u, wd);
+            if (ok && n_max > 0) {
+                ok = mbar_wait(&bars->kv_full[0], 0u, wd);
+                if (ok) {
+                    tc_fence_after();
+                    for (int t = 0; t < 2; ++t) {
+                        if (n_t[t] > 0) {
+                            issue_qk(t, 0);
+                            umma_commit(&bars->s_full[t]);
+                        }
+                    }
+                    umma_commit(&bars->kv_empty[0]);
+                }
+            }
+            for (int j = 0; ok && j < n_max; ++j) {
+                const int LV = 2 * j + 1, LK = 2 * j + 2;
+                const int sV = LV % C::kSlots, sK = LK % C::kSlots;
+                ok = mbar_wait(&bars->kv_full[sV], (uint32_t)(LV / C::kSlots) & 1u, wd);
+                if (!ok) break;
+                bool k_ready = false;
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j >= n_t[t]) continue;
+                    ok = mbar_wait(&bars->p_full[t], (uint32_t)j & 1u, wd);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(t, sV, j > 0);
+                    umma_commit(&bars->o_done[t]);
+                    if (j + 1 < n_t[t]) {
+                        if (!k_ready) {
+                            ok = mbar_wait(&bars->kv_full[sK], (uint32_t)(LK / C::kSlots) & 1u, wd);
+                            if (!ok) break;
+                            tc_fence_after();
+                            k_ready = true;
+                        }
+                        issue_qk(t, sK);
+                        umma_commit(&bars->s_full[t]);
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&bars->kv_empty[sV]);
+                if (k_ready) umma_commit(&bars->kv_empty[sK]);
+            }
+            // Drain: all MMAs issued by this thread complete before teardown.
+            umma_commit(&bars->teardown);
+            mbar_wait_drain(&bars->teardown, 0u, wd);
+        }
+        __syncwarp();
+    } else {
+        // ====================================================== softmax warpgroups
+        const int t = warp >> 2;                      // query tile 0 or 1
+        const int row = tid & (kTile - 1);            // row within the tile == TMEM lane
+        const int i = q0 + t * kTile + row;           // global query row
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + C::col_s(t);
+        const uint32_t tO = tmem + lane_base + C::col_o(t);
+        const int n = skip ? 0 : n_t[t];
+        const float c = p.scale_log2;
+        const int lim_row = p.causal ? min(kv_lim, i + 1) : kv_lim;  // visible keys: j < lim_row
+        float m_ref = -INFINITY;   // reference maximum (raw score units)
+        float l = 0.f;             // running sum of exp2((s - m_ref) * c)
+        bool ok = true;
+
+        for (int j = 0; j < n; ++j) {
+            ok = mbar_wait(&bars->s_full[t], (uint32_t)j & 1u, wd);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            float s[kTile];
+#pragma unroll
+            for (int ch = 0; ch < kTile / 32; ++ch) {
+                uint32_t r[32];
+                tmem_ld32(tS + (uint32_t)(ch * 32), r);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) s[ch * 32 + k] = __uint_as_float(r[k]);
+            }
+            tmem_wait_ld();
+            const int j0 = j * kTile;
+            if (j0 + kTile > lim_row) {
+                const int lim = lim_row - j0;
+#pragma unroll
+                for (int k = 0; k < kTile; ++k)
+                    if (k >= lim) s[k] = -INFINITY;
+            }
+            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+            for (int k = 4; k < kTile; k += 4) {
+                mx0 = fmaxf(mx0, s[k]);
+                mx1 = fmaxf(mx1, s[k + 1]);
+                mx2 = fmaxf(mx2, s[k + 2]);
+                mx3 = fmaxf(mx3, s[k + 3]);
+            }
+            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            float alpha = 1.f;
+            bool rescale = false;
+            if (m_ref == -INFINITY) {
+                m_ref = m_tile;   // first tile with a visible key: nothing accumulated yet
+            } else if ((m_tile - m_ref) * c > kRescaleLog2) {
+                alpha = fast_exp2((m_ref - m_tile) * c);
+                m_ref = m_tile;
+                l *= alpha;
+                rescale = true;
+            }
+            // P = exp2(s*c - m_ref*c), rounded to bf16 and written over S in TMEM.
+            const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+            float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < kTile / 32; ++ch) {
+                uint32_t packed[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * k], c, -mc));
+                    const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * k + 1], c, -mc));
+                    sum0 += p0;
+                    sum1 += p1;
+                    packed[k] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tS + (uint32_t)(ch * 16), packed);
+            }
+            l += sum0 + sum1;
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O holds the P.V sums of tiles < j: wait for the last of them,
+                // then bring it to the new reference maximum.
+                ok = mbar_wait(&bars->o_done[t], (uint32_t)(j - 1) & 1u, wd);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32(tO + (uint32_t)(ch * 32), r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k)
+                        r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+                    tmem_st32(tO + (uint32_t)(ch * 32), r);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[t]);
+        }
+
+        // ---------------------------------------------------- epilogue
+        if (ok && n > 0) {
+            ok = mbar_wait(&bars->o_done[t], (uint32_t)(n - 1) & 1u, wd);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) tc_fence_after();
+        }
+        const bool write = ok && !skip && (i < p.N);
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (size_t)i) * D;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[32];
+            if (ok && n > 0) {
+                tmem_ld32(tO + (uint32_t)(ch * 32), r);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) r[k] = 0u;
+            }
+            if (write) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv_l,
+                                      __uint_as_float(r[8 * v + 1]) * inv_l);
+                    w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_l,
+                                      __uint_as_float(r[8 * v + 3]) * inv_l);
+                    w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_l,
+                                      __uint_as_float(r[8 * v + 5]) * inv_l);
+                    w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_l,
+                                      __uint_as_float(r[8 * v + 7]) * inv_l);
+                    dst[v] = w;
+                }
+            }
+        }
+        if (write)
+            p.lse[(size_t)bh * p.N + (size_t)i] =
+                (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+    }
+
+    // ---------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace fa

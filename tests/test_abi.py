@@ -1,0 +1,99 @@
+"""CPU-only checks of the C-ABI library: it builds for sm_100a, loads, exports
+every symbol include/fa.h declares, and rejects bad arguments synchronously
+(these calls return before touching CUDA, so no GPU is needed)."""
+import ctypes
+import math
+
+import pytest
+
+import io_aware_exact_18_b200 as fa
+from io_aware_exact_18_b200 import build as fa_build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.load_library()
+
+
+def test_header_declares_the_boundary():
+    assert fa.declared_symbols() == ["fa_fwd", "fa_fwd_kvlen", "fa_last_device_error",
+                                     "fa_status_string"]
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(fa.LIB_PATH)
+    for name in fa.declared_symbols():
+        assert hasattr(raw, name), name
+
+
+def test_library_is_built_for_sm100a(lib):
+    log = open(fa_build.os.path.join(fa_build.PKG, "build.log")).read()
+    assert "arch=compute_100a,code=sm_100a" in log
+    assert "fa_fwd_sm100" in log  # ptxas compiled the kernel entry points
+
+
+def test_status_strings(lib):
+    assert fa.fa_status_string(fa.FA_OK) == "FA_OK"
+    for s in (fa.FA_ERR_INVALID_ARG, fa.FA_ERR_UNSUPPORTED, fa.FA_ERR_LAUNCH, fa.FA_ERR_TIMEOUT):
+        assert fa.fa_status_string(s).startswith("FA_ERR_")
+    assert fa.fa_status_string(12345) == "unknown fa status"
+
+
+# Fake, never-dereferenced device addresses: validation runs before any CUDA call.
+P = 1 << 40
+GOOD = dict(q=P, k=P + (1 << 30), v=P + (2 << 30), o=P + (3 << 30), lse=P + (4 << 30),
+            B=1, H=2, N=256, d=64, scale=0.125, causal=0)
+
+
+def call(lib, **over):
+    a = dict(GOOD, **over)
+    return lib.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"],
+                      a["d"], a["scale"], a["causal"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(B=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(H=-3), fa.FA_ERR_INVALID_ARG),
+    (dict(N=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=2), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=-0.1), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(q=0), fa.FA_ERR_INVALID_ARG),
+    (dict(lse=0), fa.FA_ERR_INVALID_ARG),
+    (dict(q=P + 8), fa.FA_ERR_INVALID_ARG),          # not 16-byte aligned
+    (dict(o=P + (3 << 30) + 2), fa.FA_ERR_INVALID_ARG),
+    (dict(lse=P + (4 << 30) + 1), fa.FA_ERR_INVALID_ARG),
+    (dict(o=P), fa.FA_ERR_INVALID_ARG),              # output aliases an input
+    (dict(lse=P + (3 << 30) + 64), fa.FA_ERR_INVALID_ARG),  # lse inside o
+    (dict(B=1 << 20, H=1 << 12), fa.FA_ERR_INVALID_ARG),    # grid too large
+])
+def test_argument_errors_are_synchronous(lib, over, status):
+    assert call(lib, **over) == status
+
+
+@pytest.mark.parametrize("over", [dict(B=0), dict(H=0), dict(N=0),
+                                  dict(B=0, q=0, k=0, v=0, o=0, lse=0)])
+def test_empty_problem_is_a_no_op(lib, over):
+    assert call(lib, **over) == fa.FA_OK
+
+
+def test_kvlen_pointer_alignment(lib):
+    a = GOOD
+    st = lib.fa_fwd_kvlen(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, 2, 256, 64, 0.125, 0,
+                          P + (5 << 30) + 2, None)
+    assert st == fa.FA_ERR_INVALID_ARG
+
+
+def test_python_wrapper_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.attention(x, x, x)
+    with pytest.raises(TypeError):
+        fa.attention(x.float(), x.float(), x.float())
+    assert math.isclose(1 / math.sqrt(64), 0.125)

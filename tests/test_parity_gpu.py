@@ -1,0 +1,194 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Tolerances (bf16 inputs, fp32 accumulation, bf16 output), per element of O
+against the oracle: max |dO| <= 2e-2 and mean |dO| <= 2e-3; for the
+log-sum-exp, |d lse| / max(|lse_ref|, 1) <= 1e-3 (the relative form is
+ill-posed where lse is near 0, e.g. causal row 0, hence the floor of 1).
+Rows with no visible key must give O = 0 and lse = -inf exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+LSE_REL = 1e-3
+
+
+def _fa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import io_aware_exact_18_b200 as fa
+    from io_aware_exact_18_b200 import build
+    build.build()
+    fa.load_library()
+    return fa
+
+
+@pytest.fixture(scope="module")
+def fa():
+    return _fa()
+
+
+def run_gpu(fa, q, k, v, causal, kv_len=None, scale=None):
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (x.to(dev).contiguous() for x in (q, k, v))
+    kvd = None if kv_len is None else kv_len.to(dev)
+    B, H, N, d = q.shape
+    out = torch.full_like(qd, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
+    fa.attention(qd, kd, vd, scale=scale, causal=causal, kv_len=kvd, out=out, lse=lse)
+    st = fa.fa_last_device_error(torch.cuda.current_stream().cuda_stream)
+    assert st == fa.FA_OK, fa.fa_status_string(st)
+    return out.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+def compare(o, lse, o_ref, lse_ref, what=""):
+    assert not np.isnan(o).any(), f"{what}: unwritten (NaN) output elements"
+    assert not np.isnan(lse).any(), f"{what}: unwritten (NaN) lse elements"
+    dead = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), dead), f"{what}: -inf pattern differs"
+    if dead.any():
+        assert np.all(o[dead] == 0.0), f"{what}: rows with no visible key must be 0"
+    err = np.abs(o - o_ref)
+    assert err.max() <= MAX_ABS, f"{what}: max|dO| = {err.max():.3e}"
+    assert err.mean() <= MEAN_ABS, f"{what}: mean|dO| = {err.mean():.3e}"
+    live = ~dead
+    if live.any():
+        rel = np.abs(lse[live] - lse_ref[live]) / np.maximum(np.abs(lse_ref[live]), 1.0)
+        assert rel.max() <= LSE_REL, f"{what}: lse rel err {rel.max():.3e}"
+    return float(err.max()), float(err.mean())
+
+
+def check_full(fa, q, k, v, causal, kv_len=None, scale=None, what=""):
+    d = q.shape[-1]
+    sc = (1.0 / math.sqrt(d)) if scale is None else scale
+    o, lse = run_gpu(fa, q, k, v, causal, kv_len, scale=sc)
+    o_ref, lse_ref = oracle.attention(q, k, v, sc, causal=causal, kv_len=kv_len)
+    return compare(o, lse, o_ref, lse_ref, what)
+
+
+# ----------------------------------------------------------------- workloads
+@pytest.mark.parametrize("idx", [1, 2, 3])
+def test_workload_full(fa, idx):
+    w = workloads.get(idx)
+    q, k, v, kv_len = workloads.make_inputs(w)
+    check_full(fa, q, k, v, w.causal, kv_len, w.scale, w.name)
+
+
+@pytest.mark.parametrize("idx", [4, 5])
+def test_workload_sampled_rows(fa, idx):
+    """Full-size launch (the one the benchmark times); the oracle evaluates a
+    seeded sample of rows in every head: first/last 64 and 64 random."""
+    w = workloads.get(idx)
+    q, k, v, kv_len = workloads.make_inputs(w)
+    o, lse = run_gpu(fa, q, k, v, w.causal, kv_len, w.scale)
+    rows = workloads.sample_rows(w.N, seed=100 + idx, n_random=64, edge=64)
+    o_ref, lse_ref = oracle.attention(q, k, v, w.scale, causal=w.causal, kv_len=kv_len,
+                                      rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], o_ref, lse_ref, w.name)
+    # properties that hold at any size, on every row
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    if w.causal:
+        v0 = v[:, :, 0].double().numpy()
+        assert np.abs(o[:, :, 0] - v0).max() <= 1e-2  # causal row 0 sees only key 0
+
+
+# ----------------------------------------------------------------- ragged / edge shapes
+RAGGED = [1, 17, 127, 128, 129, 255, 256, 257, 300, 383, 513]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", RAGGED)
+def test_ragged_lengths(fa, N, causal, d):
+    q, k, v, _ = workloads.make_custom(2, 2, N, d, seed=1000 + N + d + 7 * causal)
+    check_full(fa, q, k, v, causal, what=f"N={N} causal={causal} d={d}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_padding_edges(fa, causal, d):
+    N = 300
+    q, k, v, _ = workloads.make_custom(6, 2, N, d, seed=77 + d)
+    kv_len = torch.tensor([0, 1, 127, 128, 299, 5000], dtype=torch.int32)  # 5000 clamps to N
+    check_full(fa, q, k, v, causal, kv_len, what=f"kv_len edges causal={causal} d={d}")
+
+
+def test_peaky_rows_rescale(fa):
+    """Large |scores| (Q x 8) force many rescales of the running maximum."""
+    q, k, v, _ = workloads.make_custom(1, 4, 1024, 128, seed=9, q_mult=8.0)
+    check_full(fa, q, k, v, False, what="Qx8 non-causal")
+    check_full(fa, q, k, v, True, what="Qx8 causal")
+
+
+def test_increasing_max_forces_rescale(fa):
+    """Scores that grow along the keys: every new tile raises the row max by
+    more than the rescale threshold, so every tile rescales O."""
+    N, d = 1024, 64
+    q = torch.zeros(1, 1, N, d)
+    q[..., 0] = 1.0
+    k = torch.zeros(1, 1, N, d)
+    k[0, 0, :, 0] = torch.linspace(0, 400, N)
+    v = torch.randn(1, 1, N, d, generator=torch.Generator().manual_seed(3))
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    check_full(fa, q, k, v, False, scale=0.125, what="monotone scores")
+    check_full(fa, q, k, v, True, scale=0.125, what="monotone scores causal")
+
+
+# ----------------------------------------------------------------- pins on the GPU path
+def test_gpu_zero_query_gives_prefix_mean(fa):
+    N, d = 384, 128
+    q = torch.zeros(1, 2, N, d, dtype=torch.bfloat16)
+    _, k, v, _ = workloads.make_custom(1, 2, N, d, seed=4)
+    o, lse = run_gpu(fa, q, k, v, causal=True)
+    vv = v.double().numpy()
+    csum = np.cumsum(vv, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+    assert np.abs(o - csum).max() <= MAX_ABS
+    assert np.abs(lse - np.log(np.arange(1, N + 1))[None, None]).max() <= 1e-4
+
+
+def test_gpu_constant_values(fa):
+    q, k, _, _ = workloads.make_custom(2, 2, 257, 64, seed=5)
+    v = torch.full_like(q, 1.5)
+    o, _ = run_gpu(fa, q, k, v, causal=False)
+    assert np.abs(o - 1.5).max() == 0.0  # weights sum to 1; 1.5 is exact in bf16
+
+
+def test_deterministic(fa):
+    q, k, v, _ = workloads.make_custom(2, 4, 1000, 128, seed=8)
+    a = run_gpu(fa, q, k, v, True)
+    b = run_gpu(fa, q, k, v, True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_guard_regions_untouched(fa):
+    """O and lse live inside larger buffers; the bytes around them must
+    survive the call (no out-of-bounds writes at ragged tails)."""
+    B, H, N, d = 1, 3, 200, 128
+    q, k, v, _ = workloads.make_custom(B, H, N, d, seed=12)
+    dev = torch.device("cuda:0")
+    pad_o, pad_l = 4096, 1024
+    ob = torch.full((2 * pad_o + B * H * N * d,), 7.0, dtype=torch.bfloat16, device=dev)
+    lb = torch.full((2 * pad_l + B * H * N,), 7.0, dtype=torch.float32, device=dev)
+    out = ob[pad_o:pad_o + B * H * N * d].view(B, H, N, d)
+    lse = lb[pad_l:pad_l + B * H * N].view(B, H, N)
+    fa.attention(q.to(dev), k.to(dev), v.to(dev), causal=True, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert bool((ob[:pad_o] == 7.0).all()) and bool((ob[-pad_o:] == 7.0).all())
+    assert bool((lb[:pad_l] == 7.0).all()) and bool((lb[-pad_l:] == 7.0).all())
+
+
+def test_invalid_arguments_on_device(fa):
+    x = torch.zeros(1, 1, 128, 96, dtype=torch.bfloat16, device="cuda:0")
+    with pytest.raises(fa.FAError) as e:
+        fa.attention(x, x, x)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_last_device_error(None) == fa.FA_OK
