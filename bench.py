@@ -26,7 +26,6 @@ import hashlib
 import json
 import math
 import os
-import subprocess
 import sys
 import threading
 import time
@@ -86,68 +85,80 @@ def recorded_traffic(workload_name: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling in the background (200 ms period)."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, power and clock-event (throttle) reasons in a
+    background thread through NVML every 20 ms; read-only queries."""
+    PERIOD_S = 0.02
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.samples = []
-        self._proc = None
+    def __init__(self, torch_device_index: int):
+        self.dev = torch_device_index
+        self.samples = []          # (time, sm_mhz, max_mhz, power_w, reasons:set)
+        self._stop = threading.Event()
         self._thread = None
+        self._nvml = None
+        self._h = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        self._nvml = pynvml
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = "{:08X}:{:02X}:{:02X}.0".format(props.pci_domain_id, props.pci_bus_id,
+                                                 props.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:  # noqa: BLE001 - fall back to the visible index
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.dev]) if vis else self.dev
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
         try:
-            self._proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self._proc = None
+            self._h = self._handle()
+        except Exception:  # noqa: BLE001 - no NVML: report no samples
+            self._h = None
             return
-        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
 
-    def _read(self):
-        for line in self._proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append((time.time(), parts))
+    def _run(self):
+        n = self._nvml
+        names = {n.nvmlClocksEventReasonHwSlowdown: "hw_slowdown",
+                 n.nvmlClocksEventReasonHwThermalSlowdown: "hw_thermal_slowdown",
+                 n.nvmlClocksEventReasonSwThermalSlowdown: "sw_thermal_slowdown",
+                 n.nvmlClocksEventReasonSwPowerCap: "sw_power_cap",
+                 n.nvmlClocksEventReasonHwPowerBrakeSlowdown: "hw_power_brake_slowdown"}
+        while not self._stop.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+                mx = n.nvmlDeviceGetMaxClockInfo(self._h, n.NVML_CLOCK_SM)
+                pw = n.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                bits = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                rs = {name for bit, name in names.items() if bits & bit}
+                self.samples.append((time.time(), sm, mx, pw, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.PERIOD_S)
 
     def stop(self):
-        if self._proc is not None:
-            self._proc.terminate()
-            try:
-                self._proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self._proc.kill()
+        self._stop.set()
         if self._thread is not None:
             self._thread.join(timeout=5)
 
     def summary(self, t0, t1):
-        inside = [p for (t, p) in self.samples if t0 <= t <= t1]
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
         window = "timed"
         if len(inside) < 3:
-            inside = [p for (_, p) in self.samples]
+            inside = self.samples
             window = "warmup+timed"
         if not inside:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = sorted(v for v in (num(p[1]) for p in inside) if v is not None)
-        smax = max((v for v in (num(p[2]) for p in inside) if v is not None), default=None)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for p in inside for i in range(4)
-                          if p[5 + i].lower() == "active"})
-        pw = [v for v in (num(p[3]) for p in inside) if v is not None]
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax,
-                "reasons": reasons, "samples": len(inside), "window": window,
-                "power_w_max": max(pw) if pw else None}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable"}
+        sm = sorted(x[1] for x in inside)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": sorted(set().union(*[x[4] for x in inside])),
+                "samples": len(inside), "window": window,
+                "power_w_max": max(x[3] for x in inside), "source": "nvml, 20 ms"}
 
 
 # ----------------------------------------------------------------- CPU oracle sample
@@ -176,15 +187,16 @@ def oracle_sample_rows(w, budget_s, seed, nthreads, q, k, v, kv_len, max_rows=No
         fl = sum(4.0 * d * visible(i, b) for b in range(w.B) for i in rows) * w.H
         return dt, fl
 
-    probe = sorted(set(rng.integers(0, N, size=4).tolist()))
-    dt, fl = run(probe)
-    rate = fl / max(dt, 1e-6)
-    avg_row_flops = fl / max(len(probe), 1)
-    n_rows = int(max(4, min(N, budget_s * rate / max(avg_row_flops, 1.0))))
-    if max_rows is not None:
-        n_rows = min(n_rows, max_rows)
-    rows = sorted(set(rng.integers(0, N, size=n_rows).tolist()))
-    dt, fl = run(rows)
+    n_rows = 4
+    while True:
+        rows = sorted(set(rng.integers(0, N, size=n_rows).tolist()))
+        dt, fl = run(rows)
+        if dt >= 0.5 * budget_s or n_rows >= N or (max_rows and n_rows >= max_rows):
+            break
+        grow = 2.0 if dt <= 0 else min(8.0, max(1.5, 0.8 * budget_s / dt))
+        n_rows = int(min(N, n_rows * grow))
+        if max_rows:
+            n_rows = min(n_rows, max_rows)
     desc = (f"{len(rows)} seeded random query rows x all {w.B * w.H} (b,h) heads of "
             f"{w.name} (fraction {len(rows) / N:.4f} of the rows), fp64, "
             f"{nthreads} threads")
@@ -280,10 +292,8 @@ def our_arm(args, w):
         if st != fa.FA_OK:
             raise fa.FAError(st, "fa_fwd")
 
-    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
-                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.3)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
@@ -407,12 +417,21 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="5", help="workload index (1-5) or name")
+    ap.add_argument("--shape", default=None,
+                    help="custom B,H,N,d[,causal] (profiling of smaller cases; same recipe)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
-    w = workloads.get(args.workload)
+    if args.shape:
+        f = [int(x) for x in args.shape.split(",")]
+        B, H, N, d = f[:4]
+        causal = bool(f[4]) if len(f) > 4 else False
+        w = workloads.Workload(f"custom_B{B}_H{H}_N{N}_d{d}_{'causal' if causal else 'full'}",
+                               0, B, H, N, d, causal)
+    else:
+        w = workloads.get(args.workload)
     if args.impl == "reference":
         return reference_arm(args, w)
     return our_arm(args, w)
