@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -21,6 +22,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kWatchdogNs = 1000000000ull;  // 1 s per bounded wait
+constexpr int64_t kL2GroupBytes = 80ll << 20;     // K/V bytes of one launch-order head group
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -154,6 +156,12 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.H = H;
     p.N = N;
     p.n_pairs = (int)n_pairs;
+    // Launch-order head groups: as few groups as keep a group's K/V (2*N*d*2
+    // bytes per head) within kL2GroupBytes, with the heads split evenly.
+    const int64_t kv_head_bytes = (int64_t)N * d * 4;
+    const int64_t cap = std::max<int64_t>(1, kL2GroupBytes / kv_head_bytes);
+    const int64_t groups = (BH + cap - 1) / cap;
+    p.group_heads = (int)((BH + groups - 1) / groups);
     p.causal = causal;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.watchdog_ns = kWatchdogNs;

@@ -20,7 +20,8 @@
 //
 // Work partitioning ("FlashAttention-2 (HI)", sections 2 and 3): the grid is
 // batch x heads x (pairs of 128-row query tiles), so one long head still fills
-// every SM; the heaviest causal tiles are launched first. Inside a CTA the
+// every SM; within groups of heads whose K/V fit in L2, the heaviest causal
+// tiles are launched first. Inside a CTA the
 // work is split by role rather than by rows of the same tile:
 //   warps 0-3   softmax for query tile 0 (thread r owns row r = TMEM lane r)
 //   warps 4-7   softmax for query tile 1
@@ -75,6 +76,7 @@ struct FwdParams {
     uint32_t* dev_err;         // status word
     int B, H, N;
     int n_pairs;               // ceil(N / 256)
+    int group_heads;           // heads per L2 group (launch order)
     int causal;
     float scale_log2;          // scale * log2(e)
     uint64_t watchdog_ns;
@@ -120,8 +122,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- work unit
     // Head-major order keeps one head's K/V resident in L2 while its query
     // tiles run; within a head the heaviest (last, for causal) pair goes first.
-    const int bh = (int)(blockIdx.x / (unsigned)p.n_pairs);
-    const int pair = p.n_pairs - 1 - (int)(blockIdx.x % (unsigned)p.n_pairs);
+    // Launch order: heads are taken in groups of p.group_heads whose K/V fit
+    // in L2 together; within a group the query-tile pairs run heaviest first
+    // (the last pairs, for causal masking) across all of the group's heads, so
+    // the longest units start first and the short ones fill the tail.
+    const int BH = p.B * p.H;
+    const int per_group = p.group_heads * p.n_pairs;
+    const int grp = (int)(blockIdx.x / (unsigned)per_group);
+    const int in_grp = (int)(blockIdx.x - (unsigned)grp * (unsigned)per_group);
+    const int heads_here = min(p.group_heads, BH - grp * p.group_heads);
+    const int pair = p.n_pairs - 1 - in_grp / heads_here;
+    const int bh = grp * p.group_heads + in_grp % heads_here;
     const int b = bh / p.H;
     const int q0 = pair * 2 * kTile;
     int kv_lim = p.N;
