@@ -18,15 +18,23 @@
 // unchanged by this choice (the ratio is exact), and probabilities stay below
 // 2^8, far from fp32 or bf16 overflow.
 //
-// Work partitioning ("FlashAttention-2 (HI)", sections 2 and 3): the grid is
-// batch x heads x (pairs of 128-row query tiles), so one long head still fills
-// every SM; within groups of heads whose K/V fit in L2, the heaviest causal
-// tiles are launched first. Inside a CTA the
-// work is split by role rather than by rows of the same tile:
+// Work partitioning ("FlashAttention-2 (HI)", sections 2 and 3). A work unit
+// is one (batch, head, pair of 128-row query tiles); the grid has one CTA per
+// unit, so one long head still spreads over every SM. Units are numbered in
+// launch order: heads in groups whose K/V fit in L2 together, and within a
+// group the query-tile pairs heaviest first (the last pairs, for causal
+// masking) across the group's heads. CTAs are persistent: near the end of
+// its current unit a running CTA asks the hardware (cluster launch control)
+// to cancel the next CTA that has not started and processes that CTA's unit
+// instead, so the hardware hands out units in launch order to whichever SM
+// frees up first, the per-CTA set-up is paid once per SM, and one unit's
+// epilogue overlaps the next unit's loads and first Q.K^T.
+//
+// Roles inside a CTA (320 threads):
 //   warps 0-3   softmax for query tile 0 (thread r owns row r = TMEM lane r)
 //   warps 4-7   softmax for query tile 1
 //   warp  8     issues tcgen05 MMAs (one thread) and owns the TMEM allocation
-//   warp  9     issues TMA loads (one thread)
+//   warp  9     issues TMA loads and the unit requests (one thread)
 // With one thread per row no cross-thread reduction is needed for the row
 // max and row sum. The two softmax warpgroups ping-pong: while one works on
 // its score tile the tensor cores run the other tile's P.V and next Q.K^T.
@@ -39,6 +47,13 @@
 // Shared memory: Q0, Q1 and a ring of K/V slots, each a 128-row tile stored
 // as d/64 column blocks of 128 rows x 128 bytes in the 128-byte swizzled
 // layout that TMA writes and tcgen05 descriptors read.
+//
+// Synchronisation (mbarriers; every wait is bounded). Each barrier's phases
+// are counted per role across units; per unit and tile there is exactly one
+// q_full, q_empty and o_empty phase, max(n_t, 1) o_done phases and n_t s_full
+// and p_full phases, where n_t is the tile's number of key tiles (an idle
+// tile still takes part in its once-per-unit hand-offs), so every role can
+// compute every phase index and no barrier runs two phases ahead of a waiter.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -63,7 +78,7 @@ struct Cfg {
     static constexpr int kTileBytes = kTile * D * 2;      // one Q/K/V tile
     static constexpr int kSlots = (D == 128) ? 4 : 8;     // K/V ring depth
     static constexpr int kSmemTiles = (2 + kSlots) * kTileBytes;
-    static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 512 /*barriers*/;
+    static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 1024 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
     __device__ static constexpr uint32_t col_s(int t) { return (uint32_t)(t * 128); }
     __device__ static constexpr uint32_t col_o(int t) { return 256u + (uint32_t)(t * D); }
@@ -84,23 +99,59 @@ struct FwdParams {
 
 struct SmemBarriers {
     uint64_t q_full[2];
+    uint64_t q_empty[2];
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_done[2];
+    uint64_t o_empty[2];
+    uint64_t unit_full[2];
+    uint64_t unit_empty[2];
+    uint64_t clc_bar[2];
     uint64_t teardown;
     uint64_t kv_full[8];
     uint64_t kv_empty[8];
+    uint4 clc_resp[2];         // 16-byte aligned (offset is a multiple of 16)
+    int unit_id[2];
     uint32_t tmem_base;
     int abort;
     int skip;
 };
+static_assert(sizeof(SmemBarriers) <= 1024, "barrier region");
+static_assert(offsetof(SmemBarriers, clc_resp) % 16 == 0, "CLC response alignment");
+constexpr int kUnitConsumers = 1 + 8;  // MMA thread + one lane per softmax warp
 
-// Number of 128-key tiles query tile `t` of this CTA must visit.
+// One work unit, decoded from its launch-order index.
+struct Unit {
+    int bh, b, q0, kv_lim;
+    int n[2];                  // key tiles each query tile visits (0 = idle tile)
+    int n_max;
+};
+
+// Number of 128-key tiles a query tile starting at row q_first must visit.
 __device__ __forceinline__ int kv_tiles_for(int q_first, int N, int kv_lim, int causal) {
     if (q_first >= N) return 0;
     int lim = kv_lim;
     if (causal) lim = min(lim, q_first + kTile);
     return (lim + kTile - 1) / kTile;
+}
+
+__device__ __forceinline__ Unit decode_unit(int id, const FwdParams& p) {
+    Unit u;
+    const int BH = p.B * p.H;
+    const int per_group = p.group_heads * p.n_pairs;
+    const int grp = id / per_group;
+    const int in_grp = id - grp * per_group;
+    const int heads_here = min(p.group_heads, BH - grp * p.group_heads);
+    const int pair = p.n_pairs - 1 - in_grp / heads_here;
+    u.bh = grp * p.group_heads + in_grp % heads_here;
+    u.b = u.bh / p.H;
+    u.q0 = pair * 2 * kTile;
+    u.kv_lim = p.N;
+    if (p.kv_len != nullptr) u.kv_lim = max(0, min(p.N, p.kv_len[u.b]));
+    u.n[0] = kv_tiles_for(u.q0, p.N, u.kv_lim, p.causal);
+    u.n[1] = kv_tiles_for(u.q0 + kTile, p.N, u.kv_lim, p.causal);
+    u.n_max = max(u.n[0], u.n[1]);
+    return u;
 }
 
 template <int D>
@@ -119,37 +170,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
-    // ---------------------------------------------------------- work unit
-    // Head-major order keeps one head's K/V resident in L2 while its query
-    // tiles run; within a head the heaviest (last, for causal) pair goes first.
-    // Launch order: heads are taken in groups of p.group_heads whose K/V fit
-    // in L2 together; within a group the query-tile pairs run heaviest first
-    // (the last pairs, for causal masking) across all of the group's heads, so
-    // the longest units start first and the short ones fill the tail.
-    const int BH = p.B * p.H;
-    const int per_group = p.group_heads * p.n_pairs;
-    const int grp = (int)(blockIdx.x / (unsigned)per_group);
-    const int in_grp = (int)(blockIdx.x - (unsigned)grp * (unsigned)per_group);
-    const int heads_here = min(p.group_heads, BH - grp * p.group_heads);
-    const int pair = p.n_pairs - 1 - in_grp / heads_here;
-    const int bh = grp * p.group_heads + in_grp % heads_here;
-    const int b = bh / p.H;
-    const int q0 = pair * 2 * kTile;
-    int kv_lim = p.N;
-    if (p.kv_len != nullptr) kv_lim = max(0, min(p.N, p.kv_len[b]));
-    int n_t[2];
-    n_t[0] = kv_tiles_for(q0, p.N, kv_lim, p.causal);
-    n_t[1] = kv_tiles_for(q0 + kTile, p.N, kv_lim, p.causal);
-    const int n_max = max(n_t[0], n_t[1]);
-
     // ---------------------------------------------------------- setup
     if (tid == 0) {
-        mbar_init(&bars->q_full[0], 1);
-        mbar_init(&bars->q_full[1], 1);
         for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars->q_full[t], 1);
+            mbar_init(&bars->q_empty[t], 1);
             mbar_init(&bars->s_full[t], 1);
             mbar_init(&bars->p_full[t], kTile);
             mbar_init(&bars->o_done[t], 1);
+            mbar_init(&bars->o_empty[t], kTile);
+            mbar_init(&bars->unit_full[t], 1);
+            mbar_init(&bars->unit_empty[t], kUnitConsumers);
+            mbar_init(&bars->clc_bar[t], 1);
         }
         mbar_init(&bars->teardown, 1);
         for (int s = 0; s < C::kSlots; ++s) {
@@ -177,105 +209,184 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Watchdog wd{&bars->abort, p.dev_err, p.watchdog_ns};
 
     if (warp == kTmaWarp) {
-        // ====================================================== TMA producer
-        if (lane == 0 && !skip) {
+        // ====================================================== TMA producer + unit requests
+        if (lane == 0) {
             const uint64_t pol_kv = policy_evict_last();
             const uint64_t pol_q = policy_evict_first();
-            for (int t = 0; t < 2; ++t) {
-                if (n_t[t] == 0) continue;
-                mbar_arrive_expect_tx(&bars->q_full[t], C::kTileBytes);
-                for (int blk = 0; blk < C::kBlocks; ++blk)
-                    tma_load_3d_hint(&tm_q, &bars->q_full[t], sQ[t] + blk * C::kBlockBytes,
-                                     blk * 64, q0 + t * kTile, bh, pol_q);
-            }
-            int issued = 0;
-            for (int L = 0; L < 2 * n_max; ++L) {
+            int id = skip ? -1 : (int)blockIdx.x;
+            int L = 0;                 // K/V loads issued (K_j and V_j of every unit, in order)
+            int k = 0;                 // units published
+            int clc_pending = -1;      // slot of an unanswered cancel request
+            uint32_t clc_pending_parity = 0;
+            int q_unit[2] = {-1, -1};  // last unit whose Q tile t was requested
+            bool ok = true;
+            auto load_kv = [&](const Unit& u, int jj) -> bool {   // jj-th K/V load of unit u
                 const int slot = L % C::kSlots;
                 const uint32_t round = (uint32_t)(L / C::kSlots);
-                if (!mbar_wait(&bars->kv_empty[slot], (round & 1u) ^ 1u, wd)) break;
-                const CUtensorMap* map = (L & 1) ? &tm_v : &tm_k;
+                if (!mbar_wait(&bars->kv_empty[slot], (round & 1u) ^ 1u, wd)) return false;
+                const CUtensorMap* map = (jj & 1) ? &tm_v : &tm_k;
                 uint8_t* dst = sKV + slot * C::kTileBytes;
                 mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
                 for (int blk = 0; blk < C::kBlocks; ++blk)
                     tma_load_3d_hint(map, &bars->kv_full[slot], dst + blk * C::kBlockBytes,
-                                     blk * 64, (L >> 1) * kTile, bh, pol_kv);
-                issued = L + 1;
+                                     blk * 64, (jj >> 1) * kTile, u.bh, pol_kv);
+                ++L;
+                return true;
+            };
+            for (;; ++k) {
+                const int us = k & 1;
+                ok = mbar_wait(&bars->unit_empty[us], (uint32_t)((k >> 1) & 1) ^ 1u, wd);
+                if (!ok) break;
+                bars->unit_id[us] = id;
+                mbar_arrive(&bars->unit_full[us]);
+                if (id < 0) break;
+                const Unit u = decode_unit(id, p);
+                // K_0 and V_0 first: the ring has room while the previous unit's
+                // last tiles are consumed, and Q may have to wait for it.
+                const int early = min(2, 2 * u.n_max);
+                for (int jj = 0; ok && jj < early; ++jj) ok = load_kv(u, jj);
+                // Q tiles (one q_full phase per unit and tile, possibly with no bytes)
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (k > 0) ok = mbar_wait(&bars->q_empty[t], (uint32_t)((k - 1) & 1), wd);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars->q_full[t], u.n[t] > 0 ? C::kTileBytes : 0);
+                    q_unit[t] = k;
+                    if (u.n[t] > 0)
+                        for (int blk = 0; blk < C::kBlocks; ++blk)
+                            tma_load_3d_hint(&tm_q, &bars->q_full[t], sQ[t] + blk * C::kBlockBytes,
+                                             blk * 64, u.q0 + t * kTile, u.bh, pol_q);
+                }
+                // the rest of K_0, V_0, K_1, V_1, ... of this unit
+                for (int jj = early; ok && jj < 2 * u.n_max; ++jj) ok = load_kv(u, jj);
+                if (!ok) break;
+                // Only now (loads run about two key tiles ahead of the MMAs) ask
+                // for the next unit: a CTA takes a new unit when it is nearly
+                // free, so the heaviest remaining unit goes to the first SM that
+                // frees up, and its first loads still overlap this unit's tail.
+                mbar_arrive_expect_tx(&bars->clc_bar[us], 16);
+                clc_try_cancel(&bars->clc_resp[us], &bars->clc_bar[us]);
+                clc_pending = us;
+                clc_pending_parity = (uint32_t)((k >> 1) & 1);
+                ok = mbar_wait(&bars->clc_bar[us], clc_pending_parity, wd);
+                if (!ok) break;
+                clc_pending = -1;
+                id = clc_decode(&bars->clc_resp[us]);
+                fence_proxy_async_smem();
             }
-            // Drain: every load issued must have landed before the CTA exits.
-            for (int L = max(0, issued - C::kSlots); L < issued; ++L)
-                mbar_wait_drain(&bars->kv_full[L % C::kSlots], (uint32_t)(L / C::kSlots) & 1u,
+            // Drain: every copy issued must have landed before the CTA exits.
+            if (clc_pending >= 0) mbar_wait_drain(&bars->clc_bar[clc_pending], clc_pending_parity, wd);
+            for (int l2 = max(0, L - C::kSlots); l2 < L; ++l2)
+                mbar_wait_drain(&bars->kv_full[l2 % C::kSlots], (uint32_t)(l2 / C::kSlots) & 1u,
                                 wd);
             for (int t = 0; t < 2; ++t)
-                if (n_t[t] > 0) mbar_wait_drain(&bars->q_full[t], 0u, wd);
+                if (q_unit[t] >= 0) mbar_wait_drain(&bars->q_full[t], (uint32_t)(q_unit[t] & 1), wd);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ====================================================== MMA issuer
-        if (lane == 0 && !skip) {
+        if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTile, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+            // Descriptors are built once; a tile's start address is added in
+            // 16-byte units to the low field (addresses stay below 256 KB).
+            const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ[0]), 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(smem_u32(sKV), 16, 1024);            // K-major
+            const uint64_t dv0 = smem_desc_sw128(smem_u32(sKV), C::kBlockBytes, 1024); // MN-major
+            constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
             auto issue_qk = [&](int t, int slot) {
-                const uint32_t a0 = smem_u32(sQ[t]);
-                const uint32_t b0 = smem_u32(sKV + slot * C::kTileBytes);
+                const uint64_t a = dq0 + (uint64_t)t * kTileStep;
+                const uint64_t b = dk0 + (uint64_t)slot * kTileStep;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * C::kBlockBytes + (kk & 3) * 32);
-                    umma_ss(tmem + C::col_s(t), smem_desc_sw128(a0 + off, 16, 1024),
-                            smem_desc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t off =
+                        (uint64_t)(((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4);
+                    umma_ss(tmem + C::col_s(t), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int t, int slot, bool accumulate) {
-                const uint32_t b0 = smem_u32(sKV + slot * C::kTileBytes);
+                const uint64_t b = dv0 + (uint64_t)slot * kTileStep;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + (uint32_t)(kk * 8),
-                            smem_desc_sw128(b0 + (uint32_t)(kk * 16 * 128), C::kBlockBytes, 1024),
-                            idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                            b + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                            (accumulate || kk > 0) ? 1u : 0u);
                 }
             };
             bool ok = true;
-            for (int t = 0; t < 2 && ok; ++t)
-                if (n_t[t] > 0) ok = mbar_wait(&bars->q_full[t], 0u, wd);
-            if (ok && n_max > 0) {
-                ok = mbar_wait(&bars->kv_full[0], 0u, wd);
-                if (ok) {
-                    tc_fence_after();
-                    for (int t = 0; t < 2; ++t) {
-                        if (n_t[t] > 0) {
-                            issue_qk(t, 0);
-                            umma_commit(&bars->s_full[t]);
-                        }
-                    }
-                    umma_commit(&bars->kv_empty[0]);
-                }
-            }
-            for (int j = 0; ok && j < n_max; ++j) {
-                const int LV = 2 * j + 1, LK = 2 * j + 2;
-                const int sV = LV % C::kSlots, sK = LK % C::kSlots;
-                ok = mbar_wait(&bars->kv_full[sV], (uint32_t)(LV / C::kSlots) & 1u, wd);
+            int L0 = 0;                         // index of this unit's first K/V load
+            uint32_t ph_p[2] = {0u, 0u};        // p_full phases consumed
+            for (int k = 0; ok; ++k) {
+                const int us = k & 1;
+                ok = mbar_wait(&bars->unit_full[us], (uint32_t)((k >> 1) & 1), wd);
                 if (!ok) break;
-                bool k_ready = false;
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (j >= n_t[t]) continue;
-                    ok = mbar_wait(&bars->p_full[t], (uint32_t)j & 1u, wd);
+                const int id = bars->unit_id[us];
+                mbar_arrive(&bars->unit_empty[us]);
+                if (id < 0) break;
+                const Unit u = decode_unit(id, p);
+                // O_t is free once the previous unit's epilogue has read it
+                bool o_ready[2] = {k == 0, k == 0};
+                for (int t = 0; t < 2 && ok; ++t)
+                    ok = mbar_wait(&bars->q_full[t], (uint32_t)(k & 1), wd);
+                if (ok && u.n_max > 0) {
+                    ok = mbar_wait(&bars->kv_full[L0 % C::kSlots],
+                                   (uint32_t)(L0 / C::kSlots) & 1u, wd);
+                    if (ok) {
+                        tc_fence_after();
+                        for (int t = 0; t < 2; ++t) {
+                            if (u.n[t] > 0) {
+                                issue_qk(t, L0 % C::kSlots);
+                                umma_commit(&bars->s_full[t]);
+                                if (u.n[t] == 1) umma_commit(&bars->q_empty[t]);  // last Q.K^T
+                            }
+                        }
+                        umma_commit(&bars->kv_empty[L0 % C::kSlots]);
+                    }
+                }
+                for (int j = 0; ok && j < u.n_max; ++j) {
+                    const int LV = L0 + 2 * j + 1, LK = L0 + 2 * j + 2;
+                    const int sV = LV % C::kSlots, sK = LK % C::kSlots;
+                    ok = mbar_wait(&bars->kv_full[sV], (uint32_t)(LV / C::kSlots) & 1u, wd);
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(t, sV, j > 0);
-                    umma_commit(&bars->o_done[t]);
-                    if (j + 1 < n_t[t]) {
-                        if (!k_ready) {
-                            ok = mbar_wait(&bars->kv_full[sK], (uint32_t)(LK / C::kSlots) & 1u, wd);
-                            if (!ok) break;
-                            tc_fence_after();
-                            k_ready = true;
+                    bool k_ready = false;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j >= u.n[t]) continue;
+                        ok = mbar_wait(&bars->p_full[t], ph_p[t] & 1u, wd);
+                        ++ph_p[t];
+                        if (ok && !o_ready[t]) {
+                            ok = mbar_wait(&bars->o_empty[t], (uint32_t)((k - 1) & 1), wd);
+                            o_ready[t] = true;
                         }
-                        issue_qk(t, sK);
-                        umma_commit(&bars->s_full[t]);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(t, sV, j > 0);
+                        umma_commit(&bars->o_done[t]);
+                        if (j + 1 < u.n[t]) {
+                            if (!k_ready) {
+                                ok = mbar_wait(&bars->kv_full[sK],
+                                               (uint32_t)(LK / C::kSlots) & 1u, wd);
+                                if (!ok) break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_qk(t, sK);
+                            umma_commit(&bars->s_full[t]);
+                            if (j + 2 == u.n[t]) umma_commit(&bars->q_empty[t]);  // last Q.K^T
+                        }
                     }
+                    if (!ok) break;
+                    umma_commit(&bars->kv_empty[sV]);
+                    if (k_ready) umma_commit(&bars->kv_empty[sK]);
                 }
                 if (!ok) break;
-                umma_commit(&bars->kv_empty[sV]);
-                if (k_ready) umma_commit(&bars->kv_empty[sK]);
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (u.n[t] == 0) {                 // idle tile: its once-per-unit hand-offs
+                        umma_commit(&bars->q_empty[t]);
+                        if (!o_ready[t])
+                            ok = mbar_wait(&bars->o_empty[t], (uint32_t)((k - 1) & 1), wd);
+                        umma_commit(&bars->o_done[t]);
+                    }
+                }
+                L0 += 2 * u.n_max;
             }
             // Drain: all MMAs issued by this thread complete before teardown.
             umma_commit(&bars->teardown);
@@ -286,120 +397,141 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ====================================================== softmax warpgroups
         const int t = warp >> 2;                      // query tile 0 or 1
         const int row = tid & (kTile - 1);            // row within the tile == TMEM lane
-        const int i = q0 + t * kTile + row;           // global query row
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + C::col_s(t);
         const uint32_t tO = tmem + lane_base + C::col_o(t);
-        const int n = skip ? 0 : n_t[t];
         const float c = p.scale_log2;
-        const int lim_row = p.causal ? min(kv_lim, i + 1) : kv_lim;  // visible keys: j < lim_row
-        float m_ref = -INFINITY;   // reference maximum (raw score units)
-        float l = 0.f;             // running sum of exp2((s - m_ref) * c)
+        uint32_t ph_s = 0;     // s_full phases consumed
+        uint32_t o_base = 0;   // o_done phases of earlier units
         bool ok = true;
-
-        for (int j = 0; j < n; ++j) {
-            ok = mbar_wait(&bars->s_full[t], (uint32_t)j & 1u, wd);
+        for (int k = 0; ok; ++k) {
+            const int us = k & 1;
+            ok = mbar_wait(&bars->unit_full[us], (uint32_t)((k >> 1) & 1), wd);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            tc_fence_after();
-            float s[kTile];
-#pragma unroll
-            for (int ch = 0; ch < kTile / 32; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(tS + (uint32_t)(ch * 32), r);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) s[ch * 32 + k] = __uint_as_float(r[k]);
-            }
-            tmem_wait_ld();
-            const int j0 = j * kTile;
-            if (j0 + kTile > lim_row) {
-                const int lim = lim_row - j0;
-#pragma unroll
-                for (int k = 0; k < kTile; ++k)
-                    if (k >= lim) s[k] = -INFINITY;
-            }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-            for (int k = 4; k < kTile; k += 4) {
-                mx0 = fmaxf(mx0, s[k]);
-                mx1 = fmaxf(mx1, s[k + 1]);
-                mx2 = fmaxf(mx2, s[k + 2]);
-                mx3 = fmaxf(mx3, s[k + 3]);
-            }
-            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-            float alpha = 1.f;
-            bool rescale = false;
-            if (m_ref == -INFINITY) {
-                m_ref = m_tile;   // first tile with a visible key: nothing accumulated yet
-            } else if ((m_tile - m_ref) * c > kRescaleLog2) {
-                alpha = fast_exp2((m_ref - m_tile) * c);
-                m_ref = m_tile;
-                l *= alpha;
-                rescale = true;
-            }
-            // P = exp2(s*c - m_ref*c), rounded to bf16 and written over S in TMEM.
-            const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-            float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < kTile / 32; ++ch) {
-                uint32_t packed[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * k], c, -mc));
-                    const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * k + 1], c, -mc));
-                    sum0 += p0;
-                    sum1 += p1;
-                    packed[k] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(tS + (uint32_t)(ch * 16), packed);
-            }
-            l += sum0 + sum1;
-            if (__any_sync(0xffffffffu, rescale)) {
-                // O holds the P.V sums of tiles < j: wait for the last of them,
-                // then bring it to the new reference maximum.
-                ok = mbar_wait(&bars->o_done[t], (uint32_t)(j - 1) & 1u, wd);
+            const int id = bars->unit_id[us];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->unit_empty[us]);
+            if (id < 0) break;
+            const Unit u = decode_unit(id, p);
+            const int n = u.n[t];
+            const int i = u.q0 + t * kTile + row;     // global query row
+            const int lim_row = p.causal ? min(u.kv_lim, i + 1) : u.kv_lim;  // visible: j < lim_row
+            float m_ref = -INFINITY;   // reference maximum (raw score units)
+            float l = 0.f;             // running sum of exp2((s - m_ref) * c)
+
+            for (int j = 0; j < n; ++j) {
+                ok = mbar_wait(&bars->s_full[t], ph_s & 1u, wd);
+                ++ph_s;
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
+                float s[kTile];
+#pragma unroll
+                for (int ch = 0; ch < kTile / 32; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + (uint32_t)(ch * 32), r);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) s[ch * 32 + q] = __uint_as_float(r[q]);
+                }
+                tmem_wait_ld();
+                const int j0 = j * kTile;
+                if (j0 + kTile > lim_row) {
+                    const int lim = lim_row - j0;
+#pragma unroll
+                    for (int q = 0; q < kTile; ++q)
+                        if (q >= lim) s[q] = -INFINITY;
+                }
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int q = 4; q < kTile; q += 4) {
+                    mx0 = fmaxf(mx0, s[q]);
+                    mx1 = fmaxf(mx1, s[q + 1]);
+                    mx2 = fmaxf(mx2, s[q + 2]);
+                    mx3 = fmaxf(mx3, s[q + 3]);
+                }
+                const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                float alpha = 1.f;
+                bool rescale = false;
+                if (m_ref == -INFINITY) {
+                    m_ref = m_tile;   // first tile with a visible key: nothing accumulated yet
+                } else if ((m_tile - m_ref) * c > kRescaleLog2) {
+                    alpha = fast_exp2((m_ref - m_tile) * c);
+                    m_ref = m_tile;
+                    l *= alpha;
+                    rescale = true;
+                }
+                // P = exp2(s*c - m_ref*c), rounded to bf16 and written over S in TMEM.
+                const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+                float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+                for (int ch = 0; ch < kTile / 32; ++ch) {
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
+                        const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
+                        sum0 += p0;
+                        sum1 += p1;
+                        packed[q] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + (uint32_t)(ch * 16), packed);
+                }
+                l += sum0 + sum1;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O holds the P.V sums of tiles < j: wait for the last of them,
+                    // then bring it to the new reference maximum.
+                    ok = mbar_wait(&bars->o_done[t], (o_base + (uint32_t)(j - 1)) & 1u, wd);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t r[32];
+                        tmem_ld32(tO + (uint32_t)(ch * 32), r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
+                        tmem_st32(tO + (uint32_t)(ch * 32), r);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars->p_full[t]);
+            }
+            if (!ok) break;
+
+            // ------------------------------------------------ epilogue
+            // the unit's last o_done phase for this tile (its idle phase if n == 0)
+            const uint32_t last = o_base + (uint32_t)(n > 0 ? n - 1 : 0);
+            o_base += (uint32_t)(n > 0 ? n : 1);
+            ok = mbar_wait(&bars->o_done[t], last & 1u, wd);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const bool write = i < p.N;
+            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = p.o + ((size_t)u.bh * p.N + (size_t)i) * D;
+            uint32_t r[D];
+            if (n > 0) {
 #pragma unroll
                 for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t r[32];
-                    tmem_ld32(tO + (uint32_t)(ch * 32), r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-                    tmem_st32(tO + (uint32_t)(ch * 32), r);
+                    uint32_t* rc = r + ch * 32;
+                    tmem_ld32(tO + (uint32_t)(ch * 32), *reinterpret_cast<uint32_t(*)[32]>(rc));
                 }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full[t]);
-        }
-
-        // ---------------------------------------------------- epilogue
-        if (ok && n > 0) {
-            ok = mbar_wait(&bars->o_done[t], (uint32_t)(n - 1) & 1u, wd);
-            ok = __all_sync(0xffffffffu, ok);
-            if (ok) tc_fence_after();
-        }
-        const bool write = ok && !skip && (i < p.N);
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-        __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (size_t)i) * D;
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t r[32];
-            if (ok && n > 0) {
-                tmem_ld32(tO + (uint32_t)(ch * 32), r);
                 tmem_wait_ld();
             } else {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) r[k] = 0u;
+                for (int q = 0; q < D; ++q) r[q] = 0u;
             }
+            // O has been read: the next unit's first P.V may overwrite it
+            tc_fence_before();
+            mbar_arrive(&bars->o_empty[t]);
             if (write) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+                uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
+                for (int v = 0; v < D / 8; ++v) {
                     uint4 w;
                     w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv_l,
                                       __uint_as_float(r[8 * v + 1]) * inv_l);
@@ -411,11 +543,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       __uint_as_float(r[8 * v + 7]) * inv_l);
                     dst[v] = w;
                 }
+                p.lse[(size_t)u.bh * p.N + (size_t)i] =
+                    (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
             }
         }
-        if (write)
-            p.lse[(size_t)bh * p.N + (size_t)i] =
-                (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
     }
 
     // ---------------------------------------------------------- teardown

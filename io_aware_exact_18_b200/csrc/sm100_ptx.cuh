@@ -148,6 +148,42 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
+// ---------------------------------------------------------------- cluster launch control
+// Ask the hardware to cancel the launch of a CTA of this grid that has not
+// started yet; the 16-byte response lands in shared memory and completes
+// 16 transaction bytes on `bar`. A cancelled CTA never runs: the caller does
+// its work instead. After a failed request no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 "
+        "[%0], [%1];" ::"r"(smem_u32(resp)),
+        "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Decode a response: returns the x index of the cancelled CTA, or -1 if the
+// request failed (no CTA left to take).
+__device__ __forceinline__ int clc_decode(const void* resp) {
+    uint32_t ok, x;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "mov.u32 %1, 0;\n\t"
+        "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+        : "=r"(ok), "=r"(x)
+        : "r"(smem_u32(resp))
+        : "memory");
+    return ok ? (int)x : -1;
+}
+
+// Order this thread's generic-proxy shared-memory accesses before later
+// async-proxy ones (e.g. reusing a response buffer).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 // TMEM address: bits [31:16] lane, bits [15:0] column.
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {

@@ -122,6 +122,26 @@ def test_key_padding_edges(fa, causal, d):
     check_full(fa, q, k, v, causal, kv_len, what=f"kv_len edges causal={causal} d={d}")
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_persistent_mixed_units(fa, causal):
+    """Far more work units than SMs, so CTAs take over units of CTAs that have
+    not started; the units mix idle query tiles (N = 300 leaves the second
+    tile of the last pair empty), sequences whose keys are all hidden
+    (kv_len = 0) and short ones, so every per-unit hand-off is exercised."""
+    B, H, N, d = 40, 8, 300, 64
+    q, k, v, _ = workloads.make_custom(B, H, N, d, seed=321 + causal)
+    g = torch.Generator().manual_seed(5)
+    kv_len = torch.randint(0, N + 1, (B,), generator=g).to(torch.int32)
+    kv_len[::7] = 0
+    kv_len[1::7] = 1
+    check_full(fa, q, k, v, causal, kv_len, what=f"persistent mixed causal={causal}")
+
+
+def test_persistent_many_heads_d128(fa):
+    q, k, v, _ = workloads.make_custom(3, 100, 520, 128, seed=99)
+    check_full(fa, q, k, v, True, what="persistent 300 heads d=128")
+
+
 def test_peaky_rows_rescale(fa):
     """Large |scores| (Q x 8) force many rescales of the running maximum."""
     q, k, v, _ = workloads.make_custom(1, 4, 1024, 128, seed=9, q_mult=8.0)
