@@ -88,6 +88,19 @@ const char *fa_status_string(int status);
  */
 int fa_last_device_error(void *stream);
 
+/*
+ * Diagnostic for the kernels' failure detection (the pages have no
+ * counterpart: it checks this library's bounded waits). Launches one CTA on
+ * `stream` whose thread waits, with the same bounded-wait routine the
+ * attention kernel uses, on a shared-memory barrier that nothing completes.
+ * After limit_ns nanoseconds the wait gives up, the kernel sets the timeout
+ * bit of the device status word and returns; fa_last_device_error(stream)
+ * then reports FA_ERR_TIMEOUT (and clears the word). limit_ns must be in
+ * [1000, 5e9], else FA_ERR_INVALID_ARG. While the word is set, attention
+ * launches on the device skip their work, so read it before the next call.
+ */
+int fa_watchdog_selftest(uint64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,7 +6,8 @@ kernels of the library. There is no CPU fallback: if the library is missing
 or the device is not an sm_100 GPU, calls fail loudly.
 
 Names follow the C ABI: :func:`fa_fwd`, :func:`fa_fwd_kvlen`,
-:func:`fa_status_string`, :func:`fa_last_device_error`. :func:`attention` is
+:func:`fa_status_string`, :func:`fa_last_device_error`,
+:func:`fa_watchdog_selftest`. :func:`attention` is
 a convenience wrapper that allocates the outputs with torch and calls
 :func:`fa_fwd` / :func:`fa_fwd_kvlen` on the current stream.
 """
@@ -55,6 +56,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_error.argtypes = [vp]
     lib.fa_last_device_error.restype = i
+    lib.fa_watchdog_selftest.argtypes = [ctypes.c_uint64, vp]
+    lib.fa_watchdog_selftest.restype = i
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -87,6 +90,11 @@ def fa_status_string(status: int) -> str:
 
 def fa_last_device_error(stream) -> int:
     return load_library().fa_last_device_error(stream)
+
+
+def fa_watchdog_selftest(limit_ns: int, stream) -> int:
+    """C ABI fa_watchdog_selftest: one bounded wait that is made to run out."""
+    return load_library().fa_watchdog_selftest(int(limit_ns), stream)
 
 
 def _ptr(t):

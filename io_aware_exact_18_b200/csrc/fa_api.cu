@@ -18,6 +18,22 @@ namespace fa {
 // Per-device status word written by kernels (bit set = error seen).
 __device__ uint32_t g_dev_err = 0;
 
+// One CTA whose thread 0 waits, bounded, on a barrier nothing completes.
+__global__ void watchdog_selftest_kernel(uint32_t* dev_err, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const Watchdog wd{&abort_flag, dev_err, limit_ns};
+        (void)mbar_wait(&bar, 0u, wd);
+    }
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -202,6 +218,16 @@ FA_EXPORT const char* fa_status_string(int status) {
         case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel wait ran out of time";
         default: return "unknown fa status";
     }
+}
+
+FA_EXPORT int fa_watchdog_selftest(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1000ull || limit_ns > 5000000000ull) return FA_ERR_INVALID_ARG;
+    int dev = 0;
+    uint32_t* err = nullptr;
+    const int rc = fa::prepare_device(64, &dev, &err);
+    if (rc != FA_OK) return rc;
+    fa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_ns);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 FA_EXPORT int fa_last_device_error(void* stream) {

@@ -18,7 +18,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert fa.declared_symbols() == ["fa_fwd", "fa_fwd_kvlen", "fa_last_device_error",
-                                     "fa_status_string"]
+                                     "fa_status_string", "fa_watchdog_selftest"]
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -87,6 +87,11 @@ def test_kvlen_pointer_alignment(lib):
     st = lib.fa_fwd_kvlen(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, 2, 256, 64, 0.125, 0,
                           P + (5 << 30) + 2, None)
     assert st == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("limit", [0, 999, 5_000_000_001])
+def test_watchdog_selftest_rejects_bad_limits(lib, limit):
+    assert lib.fa_watchdog_selftest(limit, None) == fa.FA_ERR_INVALID_ARG
 
 
 def test_python_wrapper_refuses_cpu_tensors():
