@@ -12,11 +12,13 @@
 // "Online softmax"). Exponentials use base 2 with the scale folded into one
 // FFMA per score, and the division by l is deferred to the epilogue, which
 // trims the non-matmul work that "FlashAttention-2 (HI)" section 1 targets.
-// The O accumulator is rescaled only when a row maximum grows by more than
-// 2^8 (in the log2 domain); otherwise the stale maximum keeps being used as
-// the reference. Both O and l share that reference, so the final O / l is
-// unchanged by this choice (the ratio is exact), and probabilities stay below
-// 2^8, far from fp32 or bf16 overflow.
+// The reference maximum m_ref is set by a row's first key tile and is only
+// raised when a later tile's probabilities, computed against it, would sum to
+// more than 2^64: each tile is exponentiated straight away, without first
+// reducing its row maximum, and the rare tile that overshoots is redone after
+// O and l are rescaled. Both O and l share the reference, so the final O / l
+// is unchanged by this choice (the ratio is exact), and every probability
+// stays below 2^64, far inside the fp32 and bf16 range.
 //
 // Work partitioning ("FlashAttention-2 (HI)", sections 2 and 3). A work unit
 // is one (batch, head, pair of 128-row query tiles); the grid has one CTA per
@@ -67,7 +69,7 @@ constexpr int kTile = 128;         // rows per query tile and keys per KV tile
 constexpr int kThreads = 320;      // 2 softmax warpgroups + MMA warp + TMA warp
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
-constexpr float kRescaleLog2 = 8.0f;
+constexpr float kMaxTileSum = 18446744073709551616.0f;  // 2^64
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
@@ -152,6 +154,40 @@ __device__ __forceinline__ Unit decode_unit(int id, const FwdParams& p) {
     u.n[1] = kv_tiles_for(u.q0 + kTile, p.N, u.kv_lim, p.causal);
     u.n_max = max(u.n[0], u.n[1]);
     return u;
+}
+
+// Row maximum of a 128-score row held in registers.
+__device__ __forceinline__ float row_max(const float (&s)[kTile]) {
+    float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+    for (int q = 4; q < kTile; q += 4) {
+        mx0 = fmaxf(mx0, s[q]);
+        mx1 = fmaxf(mx1, s[q + 1]);
+        mx2 = fmaxf(mx2, s[q + 2]);
+        mx3 = fmaxf(mx3, s[q + 3]);
+    }
+    return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+}
+
+// P = exp2(s*c - mc), rounded to bf16 pairs and written over the row's S in
+// TMEM (warp-wide stores); returns the row sum of the fp32 probabilities.
+__device__ __forceinline__ float exp_tile(const float (&s)[kTile], float c, float mc,
+                                          uint32_t tS) {
+    float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < kTile / 32; ++ch) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
+            const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
+            sum0 += p0;
+            sum1 += p1;
+            packed[q] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + (uint32_t)(ch * 16), packed);
+    }
+    return sum0 + sum1;
 }
 
 template <int D>
@@ -442,42 +478,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int q = 0; q < kTile; ++q)
                         if (q >= lim) s[q] = -INFINITY;
                 }
-                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-                for (int q = 4; q < kTile; q += 4) {
-                    mx0 = fmaxf(mx0, s[q]);
-                    mx1 = fmaxf(mx1, s[q + 1]);
-                    mx2 = fmaxf(mx2, s[q + 2]);
-                    mx3 = fmaxf(mx3, s[q + 3]);
-                }
-                const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-                float alpha = 1.f;
+                // The first tile sets the reference maximum m_ref from its row
+                // maximum. Later tiles exponentiate against the current m_ref
+                // straight away; only if that makes the tile's row sum exceed
+                // 2^64 (some p > 2^64) does the row take its true maximum,
+                // rescale O and l, and redo the tile. Below that bound every
+                // probability, l (< N * 2^64) and O stay far inside the fp32
+                // and bf16 range, and O / l is exact whatever m_ref is.
                 bool rescale = false;
-                if (m_ref == -INFINITY) {
-                    m_ref = m_tile;   // first tile with a visible key: nothing accumulated yet
-                } else if ((m_tile - m_ref) * c > kRescaleLog2) {
-                    alpha = fast_exp2((m_ref - m_tile) * c);
-                    m_ref = m_tile;
-                    l *= alpha;
-                    rescale = true;
-                }
-                // P = exp2(s*c - m_ref*c), rounded to bf16 and written over S in TMEM.
-                const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-                float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < kTile / 32; ++ch) {
-                    uint32_t packed[16];
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
-                        const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
-                        sum0 += p0;
-                        sum1 += p1;
-                        packed[q] = pack_bf16x2(p0, p1);
+                float alpha = 1.f;
+                if (m_ref == -INFINITY) m_ref = row_max(s);
+                float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+                float l_tile = exp_tile(s, c, mc, tS);
+                const bool stale = !(l_tile <= kMaxTileSum);
+                if (__any_sync(0xffffffffu, stale)) {
+                    if (stale) {
+                        const float m_new = fmaxf(m_ref, row_max(s));
+                        alpha = fast_exp2((m_ref - m_new) * c);
+                        m_ref = m_new;
+                        l *= alpha;
+                        rescale = true;
                     }
-                    tmem_st16(tS + (uint32_t)(ch * 16), packed);
+                    mc = m_ref * c;
+                    l_tile = exp_tile(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
                 }
-                l += sum0 + sum1;
+                l += l_tile;
                 if (__any_sync(0xffffffffu, rescale)) {
                     // O holds the P.V sums of tiles < j: wait for the last of them,
                     // then bring it to the new reference maximum.

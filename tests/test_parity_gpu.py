@@ -143,10 +143,21 @@ def test_persistent_many_heads_d128(fa):
 
 
 def test_peaky_rows_rescale(fa):
-    """Large |scores| (Q x 8) force many rescales of the running maximum."""
+    """Large |scores| (Q x 8, far from the unit-normal scores the 2e-2 bound is
+    set for): rows are dominated by one or two keys, so the error is no longer
+    averaged over many weights. Its arithmetic bound: the bf16 rounding of each
+    probability (<= 2^-8 relative) moves O by at most 2^-8 * max|V|, and the
+    bf16 rounding of O adds at most 2^-8 * |O| <= 2^-8 * max|V|."""
     q, k, v, _ = workloads.make_custom(1, 4, 1024, 128, seed=9, q_mult=8.0)
-    check_full(fa, q, k, v, False, what="Qx8 non-causal")
-    check_full(fa, q, k, v, True, what="Qx8 causal")
+    bound = 2.0 ** -7 * float(v.float().abs().max())
+    for causal in (False, True):
+        o, lse = run_gpu(fa, q, k, v, causal, scale=1 / math.sqrt(128))
+        o_ref, lse_ref = oracle.attention(q, k, v, 1 / math.sqrt(128), causal=causal)
+        err = np.abs(o - o_ref)
+        assert err.max() <= bound, f"Qx8 causal={causal}: max|dO| {err.max():.3e} > {bound:.3e}"
+        assert err.mean() <= MEAN_ABS
+        rel = np.abs(lse - lse_ref) / np.maximum(np.abs(lse_ref), 1.0)
+        assert rel.max() <= LSE_REL
 
 
 def test_increasing_max_forces_rescale(fa):
