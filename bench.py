@@ -282,7 +282,11 @@ def our_arm(args, w):
     sh = stream.cuda_stream
 
     def step():
-        if kvd is None:
+        if w.kv_heads != w.H:
+            st = fa.fa_fwd_gqa(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                               lsed.data_ptr(), w.B, w.H, w.kv_heads, w.N, w.d, w.scale,
+                               int(w.causal), None if kvd is None else kvd.data_ptr(), sh)
+        elif kvd is None:
             st = fa.fa_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
                            lsed.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal), sh)
         else:
@@ -377,7 +381,8 @@ def our_arm(args, w):
                 "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
                 "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                 "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
-                "algorithmic_bytes": float(w.B * w.H * w.N * (4 * w.d * 2 + 4)),
+                "algorithmic_bytes": float(w.B * w.N * (2 * w.H * w.d * 2 + 2 * w.kv_heads * w.d * 2
+                                                        + 4 * w.H)),
                 "kernel": f"fa_fwd_sm100<{w.d}>"}
 
     cpu = None
@@ -418,7 +423,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="5", help="workload index (1-5) or name")
     ap.add_argument("--shape", default=None,
-                    help="custom B,H,N,d[,causal] (profiling of smaller cases; same recipe)")
+                    help="custom B,H,N,d[,causal[,H_kv]] (smaller or grouped-query cases; "
+                         "same recipe)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -428,8 +434,10 @@ def main(argv=None):
         f = [int(x) for x in args.shape.split(",")]
         B, H, N, d = f[:4]
         causal = bool(f[4]) if len(f) > 4 else False
-        w = workloads.Workload(f"custom_B{B}_H{H}_N{N}_d{d}_{'causal' if causal else 'full'}",
-                               0, B, H, N, d, causal)
+        H_kv = f[5] if len(f) > 5 else None
+        tag = "" if H_kv is None else f"_Hkv{H_kv}"
+        w = workloads.Workload(f"custom_B{B}_H{H}{tag}_N{N}_d{d}_{'causal' if causal else 'full'}",
+                               0, B, H, N, d, causal, H_kv=H_kv)
     else:
         w = workloads.get(args.workload)
     if args.impl == "reference":

@@ -76,6 +76,19 @@ int fa_fwd_kvlen(const void *q, const void *k, const void *v, void *o, float *ls
                  int B, int H, int N, int d, float scale, int causal,
                  const int32_t *kv_len, void *stream);
 
+/*
+ * Grouped- and multi-query attention (the FlashAttention-2 extension to
+ * multi-query attention, "FlashAttention (UR)", section "FlashAttention-2
+ * (2023)"): q, o are bf16 [B, H, N, d] and lse fp32 [B, H, N] as above, but
+ * k, v are bf16 [B, H_kv, N, d] with H a multiple of H_kv; query head h
+ * attends with K/V head h / (H / H_kv). H_kv == H is fa_fwd_kvlen; H_kv == 1
+ * is multi-query attention. kv_len as in fa_fwd_kvlen (nullable). H_kv < 1,
+ * H_kv > H or H % H_kv != 0 returns FA_ERR_INVALID_ARG.
+ */
+int fa_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse,
+               int B, int H, int H_kv, int N, int d, float scale, int causal,
+               const int32_t *kv_len, void *stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(int status);
 

@@ -5,11 +5,11 @@ Every function here only marshals arguments; all arithmetic runs in the CUDA
 kernels of the library. There is no CPU fallback: if the library is missing
 or the device is not an sm_100 GPU, calls fail loudly.
 
-Names follow the C ABI: :func:`fa_fwd`, :func:`fa_fwd_kvlen`,
+Names follow the C ABI: :func:`fa_fwd`, :func:`fa_fwd_kvlen`, :func:`fa_fwd_gqa`,
 :func:`fa_status_string`, :func:`fa_last_device_error`,
-:func:`fa_watchdog_selftest`. :func:`attention` is
-a convenience wrapper that allocates the outputs with torch and calls
-:func:`fa_fwd` / :func:`fa_fwd_kvlen` on the current stream.
+:func:`fa_watchdog_selftest`. :func:`attention` is a convenience wrapper that
+allocates the outputs with torch and calls :func:`fa_fwd` / :func:`fa_fwd_kvlen`
+/ :func:`fa_fwd_gqa` on the current stream.
 """
 from __future__ import annotations
 
@@ -52,6 +52,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd.restype = i
     lib.fa_fwd_kvlen.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
     lib.fa_fwd_kvlen.restype = i
+    lib.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp]
+    lib.fa_fwd_gqa.restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_error.argtypes = [vp]
@@ -81,6 +83,12 @@ def fa_fwd_kvlen(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, stream) -> 
                                        kv_len, stream)
 
 
+def fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, kv_len, stream) -> int:
+    """C ABI fa_fwd_gqa: k, v have H_kv heads shared by groups of H / H_kv query heads."""
+    return load_library().fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal,
+                                     kv_len, stream)
+
+
 def fa_status_string(status: int) -> str:
     try:
         return load_library().fa_status_string(int(status)).decode()
@@ -103,7 +111,9 @@ def _ptr(t):
 
 def attention(q, k, v, scale=None, causal=False, kv_len=None, out=None, lse=None,
               stream=None, check=True):
-    """O, lse = attention(q, k, v) for bf16 CUDA tensors [B, H, N, d].
+    """O, lse = attention(q, k, v) for bf16 CUDA tensors q [B, H, N, d] and
+    k, v [B, H_kv, N, d] (H_kv == H, or H a multiple of H_kv for grouped /
+    multi-query attention).
 
     Allocates O (bf16) and lse (fp32) unless given, calls the C ABI on the
     current torch stream (or `stream`), and raises FAError on a bad status.
@@ -113,8 +123,10 @@ def attention(q, k, v, scale=None, causal=False, kv_len=None, out=None, lse=None
         raise TypeError("q, k, v must be bfloat16")
     if not (q.is_cuda and k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be CUDA tensors (no CPU fallback)")
-    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
-        raise ValueError(f"q, k, v must share one [B,H,N,d] shape, got {q.shape} {k.shape} {v.shape}")
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape or \
+            (q.shape[0], q.shape[2], q.shape[3]) != (k.shape[0], k.shape[2], k.shape[3]):
+        raise ValueError(f"q [B,H,N,d] and k, v [B,H_kv,N,d] expected, got "
+                         f"{q.shape} {k.shape} {v.shape}")
     if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
         raise ValueError("q, k, v must be contiguous")
     B, H, N, d = q.shape
@@ -125,12 +137,17 @@ def attention(q, k, v, scale=None, causal=False, kv_len=None, out=None, lse=None
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     s = stream if stream is not None else torch.cuda.current_stream(q.device).cuda_stream
-    if kv_len is None:
+    H_kv = k.shape[1]
+    if kv_len is not None and (kv_len.dtype != torch.int32 or not kv_len.is_cuda
+                               or kv_len.shape != (B,)):
+        raise ValueError("kv_len must be a CUDA int32 tensor of shape [B]")
+    if H_kv != H:
+        st = fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, N, d,
+                        float(scale), int(bool(causal)), _ptr(kv_len), s)
+    elif kv_len is None:
         st = fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
                     float(scale), int(bool(causal)), s)
     else:
-        if kv_len.dtype != torch.int32 or not kv_len.is_cuda or kv_len.shape != (B,):
-            raise ValueError("kv_len must be a CUDA int32 tensor of shape [B]")
         st = fa_fwd_kvlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
                           float(scale), int(bool(causal)), _ptr(kv_len), s)
     if check and st != FA_OK:

@@ -128,9 +128,11 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int N, int d, float scale, int causal, const int32_t* kv_len, void* stream) {
+             int H_kv, int N, int d, float scale, int causal, const int32_t* kv_len,
+             void* stream) {
     // ---- arguments (synchronous, nothing launched on error)
     if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+    if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -142,14 +144,16 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
         return FA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0) return FA_ERR_INVALID_ARG;
     const int64_t BH = (int64_t)B * H;
+    const int64_t BHkv = (int64_t)B * H_kv;
     const int64_t n_pairs = ((int64_t)N + 255) / 256;
     if (BH > INT32_MAX || BH * n_pairs > INT32_MAX) return FA_ERR_INVALID_ARG;
     const size_t elems = (size_t)BH * (size_t)N * (size_t)d;
     if ((double)BH * N * d > 9.0e18) return FA_ERR_INVALID_ARG;
     const size_t tbytes = elems * 2, lbytes = (size_t)BH * (size_t)N * 4;
-    if (overlaps(o, tbytes, q, tbytes) || overlaps(o, tbytes, k, tbytes) ||
-        overlaps(o, tbytes, v, tbytes) || overlaps(lse, lbytes, q, tbytes) ||
-        overlaps(lse, lbytes, k, tbytes) || overlaps(lse, lbytes, v, tbytes) ||
+    const size_t kvbytes = (size_t)BHkv * (size_t)N * (size_t)d * 2;
+    if (overlaps(o, tbytes, q, tbytes) || overlaps(o, tbytes, k, kvbytes) ||
+        overlaps(o, tbytes, v, kvbytes) || overlaps(lse, lbytes, q, tbytes) ||
+        overlaps(lse, lbytes, k, kvbytes) || overlaps(lse, lbytes, v, kvbytes) ||
         overlaps(lse, lbytes, o, tbytes))
         return FA_ERR_INVALID_ARG;
 
@@ -160,8 +164,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 
     alignas(64) CUtensorMap mq, mk, mv;
     if ((rc = make_map(&mq, q, (int)BH, N, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mk, k, (int)BH, N, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, v, (int)BH, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, k, (int)BHkv, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, v, (int)BHkv, N, d)) != FA_OK) return rc;
 
     FwdParams p{};
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -170,12 +174,14 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.dev_err = err;
     p.B = B;
     p.H = H;
+    p.H_kv = H_kv;
     p.N = N;
     p.n_pairs = (int)n_pairs;
     // Launch-order head groups: as few groups as keep a group's K/V (2*N*d*2
-    // bytes per head) within kL2GroupBytes, with the heads split evenly.
+    // bytes per K/V head, shared by H / H_kv query heads) within
+    // kL2GroupBytes, with the query heads split evenly.
     const int64_t kv_head_bytes = (int64_t)N * d * 4;
-    const int64_t cap = std::max<int64_t>(1, kL2GroupBytes / kv_head_bytes);
+    const int64_t cap = std::max<int64_t>(1, kL2GroupBytes / kv_head_bytes) * (H / H_kv);
     const int64_t groups = (BH + cap - 1) / cap;
     p.group_heads = (int)((BH + groups - 1) / groups);
     p.causal = causal;
@@ -200,13 +206,19 @@ extern "C" {
 
 FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
            int d, float scale, int causal, void* stream) {
-    return fa::fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, nullptr, stream);
+    return fa::fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, nullptr, stream);
 }
 
 FA_EXPORT int fa_fwd_kvlen(const void* q, const void* k, const void* v, void* o, float* lse,
                            int B, int H, int N, int d, float scale, int causal,
                            const int32_t* kv_len, void* stream) {
-    return fa::fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, kv_len, stream);
+    return fa::fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, kv_len, stream);
+}
+
+FA_EXPORT int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int H_kv, int N, int d, float scale, int causal,
+                         const int32_t* kv_len, void* stream) {
+    return fa::fwd_impl(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, kv_len, stream);
 }
 
 FA_EXPORT const char* fa_status_string(int status) {

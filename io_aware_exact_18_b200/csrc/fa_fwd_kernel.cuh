@@ -32,6 +32,12 @@
 // frees up first, the per-CTA set-up is paid once per SM, and one unit's
 // epilogue overlaps the next unit's loads and first Q.K^T.
 //
+// Grouped / multi-query attention (the FlashAttention-2 extension to MQA,
+// "FlashAttention (UR)", section "FlashAttention-2 (2023)"): K and V may have
+// H_kv heads shared by groups of H / H_kv query heads; a unit's K/V tiles come
+// from its query head's group head, and neighbouring query heads (same group)
+// run next to each other so the shared K/V stays in L2.
+//
 // Roles inside a CTA (320 threads):
 //   warps 0-3   softmax for query tile 0 (thread r owns row r = TMEM lane r)
 //   warps 4-7   softmax for query tile 1
@@ -92,6 +98,7 @@ struct FwdParams {
     const int32_t* kv_len;     // [B] or nullptr
     uint32_t* dev_err;         // status word
     int B, H, N;
+    int H_kv;                  // K/V heads; query head h reads K/V head h / (H / H_kv)
     int n_pairs;               // ceil(N / 256)
     int group_heads;           // heads per L2 group (launch order)
     int causal;
@@ -125,6 +132,7 @@ constexpr int kUnitConsumers = 1 + 8;  // MMA thread + one lane per softmax warp
 // One work unit, decoded from its launch-order index.
 struct Unit {
     int bh, b, q0, kv_lim;
+    int bkv;                   // K/V head row in the [B*H_kv, N, d] view
     int n[2];                  // key tiles each query tile visits (0 = idle tile)
     int n_max;
 };
@@ -147,6 +155,7 @@ __device__ __forceinline__ Unit decode_unit(int id, const FwdParams& p) {
     const int pair = p.n_pairs - 1 - in_grp / heads_here;
     u.bh = grp * p.group_heads + in_grp % heads_here;
     u.b = u.bh / p.H;
+    u.bkv = u.b * p.H_kv + (u.bh - u.b * p.H) / (p.H / p.H_kv);
     u.q0 = pair * 2 * kTile;
     u.kv_lim = p.N;
     if (p.kv_len != nullptr) u.kv_lim = max(0, min(p.N, p.kv_len[u.b]));
@@ -265,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
                 for (int blk = 0; blk < C::kBlocks; ++blk)
                     tma_load_3d_hint(map, &bars->kv_full[slot], dst + blk * C::kBlockBytes,
-                                     blk * 64, (jj >> 1) * kTile, u.bh, pol_kv);
+                                     blk * 64, (jj >> 1) * kTile, u.bkv, pol_kv);
                 ++L;
                 return true;
             };

@@ -49,6 +49,13 @@ def _bind(lib):
                                      c_int, c_int, c_double, c_int, i32p, i32p,
                                      c_int, c_int]
     lib.oracle_attn_bf16.restype = c_int
+    lib.oracle_attn_gqa_f64.argtypes = [dp, dp, dp, dp, dp, c_int, c_int, c_int, c_int,
+                                        c_int, c_double, c_int, i32p, c_int]
+    lib.oracle_attn_gqa_f64.restype = c_int
+    lib.oracle_attn_gqa_bf16.argtypes = [u16p, u16p, u16p, dp, dp, c_int, c_int, c_int,
+                                         c_int, c_int, c_double, c_int, i32p, i32p, c_int,
+                                         c_int]
+    lib.oracle_attn_gqa_bf16.restype = c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     return lib
@@ -93,8 +100,10 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
               nthreads=0, lib=None):
     """Exact attention in fp64.
 
-    q, k, v: [B, H, N, d] as torch bf16 / float tensors or numpy arrays
-    (uint16 arrays are read as bf16 bit patterns). kv_len: None or [B] ints.
+    q: [B, H, N, d]; k, v: [B, Hkv, N, d] with H a multiple of Hkv (query head
+    h uses K/V head h // (H // Hkv); Hkv == H is plain multi-head attention),
+    as torch bf16 / float tensors or numpy arrays (uint16 arrays are read as
+    bf16 bit patterns). kv_len: None or [B] ints.
     rows: None (all rows) or a list of query-row indices evaluated in every
     (b, h). Returns (o [B,H,R,d] float64, lse [B,H,R] float64), R = N or
     len(rows).
@@ -105,9 +114,12 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
     va, vb16 = _as_numpy(v)
     if not (qb16 == kb16 == vb16):
         raise TypeError("q, k, v must share one element type")
-    if qa.ndim != 4 or qa.shape != ka.shape or qa.shape != va.shape:
+    if qa.ndim != 4 or ka.shape != va.shape or ka.ndim != 4:
         raise ValueError(f"bad shapes {qa.shape} {ka.shape} {va.shape}")
     B, H, N, d = qa.shape
+    Hkv = ka.shape[1]
+    if ka.shape != (B, Hkv, N, d) or Hkv < 1 or H % Hkv:
+        raise ValueError(f"bad shapes {qa.shape} {ka.shape} {va.shape}")
     kvp = None
     if kv_len is not None:
         kvl = np.ascontiguousarray(np.asarray(
@@ -126,17 +138,17 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
             ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
             rp = ra.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
         u16p = ctypes.POINTER(ctypes.c_uint16)
-        rc = lib.oracle_attn_bf16(qa.ctypes.data_as(u16p), ka.ctypes.data_as(u16p),
-                                  va.ctypes.data_as(u16p), o.ctypes.data_as(dp),
-                                  lse.ctypes.data_as(dp), B, H, N, d, float(scale),
-                                  int(bool(causal)), kvp, rp, R, int(nthreads))
+        rc = lib.oracle_attn_gqa_bf16(qa.ctypes.data_as(u16p), ka.ctypes.data_as(u16p),
+                                      va.ctypes.data_as(u16p), o.ctypes.data_as(dp),
+                                      lse.ctypes.data_as(dp), B, H, Hkv, N, d, float(scale),
+                                      int(bool(causal)), kvp, rp, R, int(nthreads))
     else:
         if rows is not None:
             raise ValueError("row subsets are supported for bf16 inputs only")
-        rc = lib.oracle_attn_f64(qa.ctypes.data_as(dp), ka.ctypes.data_as(dp),
-                                 va.ctypes.data_as(dp), o.ctypes.data_as(dp),
-                                 lse.ctypes.data_as(dp), B, H, N, d, float(scale),
-                                 int(bool(causal)), kvp, int(nthreads))
+        rc = lib.oracle_attn_gqa_f64(qa.ctypes.data_as(dp), ka.ctypes.data_as(dp),
+                                     va.ctypes.data_as(dp), o.ctypes.data_as(dp),
+                                     lse.ctypes.data_as(dp), B, H, Hkv, N, d, float(scale),
+                                     int(bool(causal)), kvp, int(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle returned error {rc}")
     return o, lse

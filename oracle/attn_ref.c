@@ -15,6 +15,11 @@
  * materialised, then the softmax is taken in two passes (max, then sum of
  * exponentials) over the whole row. No tiling, no online rescaling.
  *
+ * Grouped / multi-query attention (the FlashAttention-2 extension to MQA named
+ * in "FlashAttention (UR)", section "FlashAttention-2 (2023)"): K and V may
+ * have Hkv <= H heads, H a multiple of Hkv; query head h attends with K/V head
+ * h / (H / Hkv). Hkv == H is ordinary multi-head attention.
+ *
  * Readings taken where the pages are silent:
  *   - scale is passed by the caller (1/sqrt(d) in every workload);
  *   - the mask is additive -inf; causal means key j is allowed iff j <= i
@@ -113,12 +118,14 @@ static int check_args(int B, int H, int N, int d, double scale, int causal)
  */
 static int attn_driver(const double *qd, const double *kd, const double *vd,
                        const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
-                       double *o, double *lse, int B, int H, int N, int d,
+                       double *o, double *lse, int B, int H, int Hkv, int N, int d,
                        double scale, int causal, const int32_t *kv_len,
                        const int32_t *rows, int nrows, int nthreads)
 {
     int rc = check_args(B, H, N, d, scale, causal);
     if (rc) return rc;
+    if (B == 0 || H == 0) return ORACLE_OK;
+    if (Hkv <= 0 || Hkv > H || H % Hkv != 0) return ORACLE_EINVAL;
     if (nrows < 0 || (rows == NULL && nrows != N)) return ORACLE_EINVAL;
     if (rows)
         for (int r = 0; r < nrows; ++r)
@@ -152,17 +159,18 @@ static int attn_driver(const double *qd, const double *kd, const double *vd,
             if (kv_lim > N) kv_lim = N;
         }
         for (int h = 0; h < H; ++h) {
-            const size_t base = ((size_t)b * H + h) * head;
+            const size_t base = ((size_t)b * H + h) * head;                  /* Q, O */
+            const size_t kvbase = ((size_t)b * Hkv + h / (H / Hkv)) * head;  /* K, V */
             const double *Q, *K, *V;
             if (widen) {
                 for (size_t e = 0; e < head; ++e) {
                     Qh[e] = bf16_to_f64(qb[base + e]);
-                    Kh[e] = bf16_to_f64(kb[base + e]);
-                    Vh[e] = bf16_to_f64(vb[base + e]);
+                    Kh[e] = bf16_to_f64(kb[kvbase + e]);
+                    Vh[e] = bf16_to_f64(vb[kvbase + e]);
                 }
                 Q = Qh; K = Kh; V = Vh;
             } else {
-                Q = qd + base; K = kd + base; V = vd + base;
+                Q = qd + base; K = kd + kvbase; V = vd + kvbase;
             }
             double *o_bh = o + ((size_t)b * H + h) * (size_t)nrows * d;
             double *l_bh = lse + ((size_t)b * H + h) * (size_t)nrows;
@@ -196,7 +204,7 @@ int oracle_attn_f64(const double *q, const double *k, const double *v,
                     int nthreads)
 {
     if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, N, d, scale,
+    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, H, N, d, scale,
                        causal, kv_len, NULL, N, nthreads);
 }
 
@@ -207,7 +215,27 @@ int oracle_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *rows, int nrows, int nthreads)
 {
     if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, N, d, scale,
+    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, H, N, d, scale,
+                       causal, kv_len, rows, nrows, nthreads);
+}
+
+/* Grouped/multi-query forms: q, o [B,H,N,d]; k, v [B,Hkv,N,d]. */
+int oracle_attn_gqa_f64(const double *q, const double *k, const double *v,
+                        double *o, double *lse, int B, int H, int Hkv, int N, int d,
+                        double scale, int causal, const int32_t *kv_len, int nthreads)
+{
+    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
+    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, Hkv, N, d, scale,
+                       causal, kv_len, NULL, N, nthreads);
+}
+
+int oracle_attn_gqa_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         double *o, double *lse, int B, int H, int Hkv, int N, int d,
+                         double scale, int causal, const int32_t *kv_len,
+                         const int32_t *rows, int nrows, int nthreads)
+{
+    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
+    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, Hkv, N, d, scale,
                        causal, kv_len, rows, nrows, nthreads);
 }
 

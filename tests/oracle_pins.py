@@ -220,6 +220,29 @@ def pin_no_visible_key(lib):
     assert np.all(np.isfinite(lse[1]))
 
 
+def pin_grouped_heads_equal_repeated_heads(lib):
+    """Grouped/multi-query attention is multi-head attention whose K/V heads are
+    repeated for each group of query heads (query head h uses K/V head
+    h // (H // Hkv)); with Hkv == H nothing changes."""
+    rng = np.random.default_rng(20)
+    B, H, N, d = 2, 6, 23, 8
+    q = rng.standard_normal((B, H, N, d))
+    for Hkv in (1, 2, 3, 6):
+        k = rng.standard_normal((B, Hkv, N, d))
+        v = rng.standard_normal((B, Hkv, N, d))
+        g = H // Hkv
+        k_rep = np.repeat(k, g, axis=1)
+        v_rep = np.repeat(v, g, axis=1)
+        for causal, kvl in [(False, None), (True, [23, 9])]:
+            o, lse = _attn(lib, q, k, v, 0.3, causal, kvl)
+            o2, l2 = _attn(lib, q, k_rep, v_rep, 0.3, causal, kvl)
+            assert np.array_equal(o, o2) and np.array_equal(lse, l2), (Hkv, causal)
+            if Hkv == 1:   # every query head sees the same keys: permuting heads commutes
+                perm = rng.permutation(H)
+                o3, _ = _attn(lib, q[:, perm], k, v, 0.3, causal, kvl)
+                assert np.allclose(o3, o[:, perm], atol=TOL, rtol=0)
+
+
 ALL_PINS = [
     pin_golden_closed_forms,
     pin_rows_sum_to_one,
@@ -231,6 +254,7 @@ ALL_PINS = [
     pin_torch_sdpa,
     pin_online_equals_full,
     pin_no_visible_key,
+    pin_grouped_heads_equal_repeated_heads,
 ]
 
 

@@ -17,8 +17,9 @@ def lib():
 
 
 def test_header_declares_the_boundary():
-    assert fa.declared_symbols() == ["fa_fwd", "fa_fwd_kvlen", "fa_last_device_error",
-                                     "fa_status_string", "fa_watchdog_selftest"]
+    assert fa.declared_symbols() == ["fa_fwd", "fa_fwd_gqa", "fa_fwd_kvlen",
+                                     "fa_last_device_error", "fa_status_string",
+                                     "fa_watchdog_selftest"]
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -87,6 +88,18 @@ def test_kvlen_pointer_alignment(lib):
     st = lib.fa_fwd_kvlen(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, 2, 256, 64, 0.125, 0,
                           P + (5 << 30) + 2, None)
     assert st == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("H,H_kv,status", [(8, 0, fa.FA_ERR_INVALID_ARG),
+                                            (8, 3, fa.FA_ERR_INVALID_ARG),
+                                            (8, 16, fa.FA_ERR_INVALID_ARG),
+                                            (8, -1, fa.FA_ERR_INVALID_ARG),
+                                            (0, 0, fa.FA_OK)])
+def test_gqa_head_arguments(lib, H, H_kv, status):
+    a = GOOD
+    st = lib.fa_fwd_gqa(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, H, H_kv, 256, 64, 0.125,
+                        0, None, None)
+    assert st == status
 
 
 @pytest.mark.parametrize("limit", [0, 999, 5_000_000_001])

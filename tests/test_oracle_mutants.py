@@ -31,6 +31,8 @@ MUTANTS = {
     "unnormalised_weights": ("double p = exp(srow[j] - lse);",
                              "double p = exp(srow[j] - m);"),
     "max_not_subtracted_in_sum": ("sum += exp(srow[j] - m);", "sum += exp(srow[j]);"),
+    "kv_head_modulo_instead_of_group": ("h / (H / Hkv)) * head;  /* K, V */",
+                                        "h % Hkv) * head;  /* K, V */"),
 }
 
 

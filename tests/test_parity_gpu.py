@@ -142,6 +142,21 @@ def test_persistent_many_heads_d128(fa):
     check_full(fa, q, k, v, True, what="persistent 300 heads d=128")
 
 
+@pytest.mark.parametrize("H,H_kv", [(8, 2), (6, 1), (4, 4)])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_grouped_and_multi_query(fa, H, H_kv, d, causal):
+    """K/V heads shared by groups of query heads (H_kv = 1: multi-query)."""
+    B, N = 3, 333
+    g = torch.Generator().manual_seed(1000 + H * 10 + H_kv + d + causal)
+    q = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+    kv_len = torch.tensor([333, 200, 0], dtype=torch.int32)
+    check_full(fa, q, k, v, causal, kv_len, what=f"H={H} H_kv={H_kv} d={d} causal={causal}")
+    check_full(fa, q, k, v, causal, None, what=f"H={H} H_kv={H_kv} d={d} causal={causal}")
+
+
 def test_peaky_rows_rescale(fa):
     """Large |scores| (Q x 8, far from the unit-normal scores the 2e-2 bound is
     set for): rows are dominated by one or two keys, so the error is no longer

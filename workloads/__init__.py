@@ -12,7 +12,8 @@ dataset is involved: every tensor is i.i.d. N(0, 1) rounded to bfloat16.
 
 Recipe (fixed, so any run can be reproduced):
   * generator: ``torch.Generator('cpu').manual_seed(seed)``;
-  * draw order: Q, then K, then V, each ``torch.randn([B, H, N, d])`` in fp32,
+  * draw order: Q, then K, then V, each ``torch.randn`` in fp32 of shape
+    ``[B, H, N, d]`` (K and V: ``[B, H_kv, N, d]`` for grouped-query shapes),
     then ``.to(torch.bfloat16)`` (round to nearest even);
   * ``q_mult`` (long-range case): Q is multiplied by 4 after rounding, which is
     exact in bf16 because 4 is a power of two;
@@ -40,6 +41,11 @@ class Workload:
     causal: bool
     q_mult: float = 1.0
     kv_len_range: Optional[tuple] = None  # (lo, hi) inclusive, or None
+    H_kv: Optional[int] = None            # K/V heads (grouped/multi-query); None = H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.H_kv is None else self.H_kv
 
     @property
     def scale(self) -> float:
@@ -58,7 +64,7 @@ class Workload:
     def describe(self) -> dict:
         return {
             "workload": self.name,
-            "B": self.B, "H": self.H, "N": self.N, "d": self.d,
+            "B": self.B, "H": self.H, "H_kv": self.kv_heads, "N": self.N, "d": self.d,
             "causal": self.causal,
             "mask": ("causal" if self.causal else
                      ("key_padding" if self.kv_len_range else "none")),
@@ -90,13 +96,15 @@ def get(key) -> Workload:
 
 
 def make_inputs(w: Workload, seed: Optional[int] = None):
-    """Return (q, k, v, kv_len) on the CPU; q/k/v bf16 [B,H,N,d], kv_len int32 [B] or None."""
+    """Return (q, k, v, kv_len) on the CPU; q bf16 [B,H,N,d], k/v bf16
+    [B,H_kv,N,d] (H_kv = H unless grouped), kv_len int32 [B] or None."""
     g = torch.Generator(device="cpu")
     g.manual_seed(w.index if seed is None else seed)
     shape = (w.B, w.H, w.N, w.d)
+    kv_shape = (w.B, w.kv_heads, w.N, w.d)
     q = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
-    k = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
-    v = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
     if w.q_mult != 1.0:
         q = q * w.q_mult
     kv_len = None
