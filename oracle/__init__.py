@@ -56,6 +56,10 @@ def _bind(lib):
                                          c_int, c_int, c_double, c_int, i32p, i32p, c_int,
                                          c_int]
     lib.oracle_attn_gqa_bf16.restype = c_int
+    lib.oracle_attn_general.argtypes = [dp, dp, dp, u16p, u16p, u16p, dp, dp, c_int, c_int,
+                                         c_int, c_int, c_int, c_int, c_double, c_int, i32p,
+                                         i32p, c_int, c_int]
+    lib.oracle_attn_general.restype = c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     return lib
@@ -100,13 +104,14 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
               nthreads=0, lib=None):
     """Exact attention in fp64.
 
-    q: [B, H, N, d]; k, v: [B, Hkv, N, d] with H a multiple of Hkv (query head
-    h uses K/V head h // (H // Hkv); Hkv == H is plain multi-head attention),
-    as torch bf16 / float tensors or numpy arrays (uint16 arrays are read as
-    bf16 bit patterns). kv_len: None or [B] ints.
-    rows: None (all rows) or a list of query-row indices evaluated in every
-    (b, h). Returns (o [B,H,R,d] float64, lse [B,H,R] float64), R = N or
-    len(rows).
+    q: [B, H, Nq, d]; k, v: [B, Hkv, Nk, d] with H a multiple of Hkv (query
+    head h uses K/V head h // (H // Hkv); Hkv == H is plain multi-head
+    attention) and Nq <= Nk (query row i stands at key position i + Nk - Nq;
+    Nq == Nk is ordinary self-attention), as torch bf16 / float tensors or
+    numpy arrays (uint16 arrays are read as bf16 bit patterns). kv_len: None
+    or [B] ints. rows: None (all rows) or a list of query-row indices
+    evaluated in every (b, h). Returns (o [B,H,R,d] float64, lse [B,H,R]
+    float64), R = Nq or len(rows).
     """
     lib = lib or load()
     qa, qb16 = _as_numpy(q)
@@ -116,9 +121,9 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
         raise TypeError("q, k, v must share one element type")
     if qa.ndim != 4 or ka.shape != va.shape or ka.ndim != 4:
         raise ValueError(f"bad shapes {qa.shape} {ka.shape} {va.shape}")
-    B, H, N, d = qa.shape
-    Hkv = ka.shape[1]
-    if ka.shape != (B, Hkv, N, d) or Hkv < 1 or H % Hkv:
+    B, H, Nq, d = qa.shape
+    Hkv, N = ka.shape[1], ka.shape[2]
+    if ka.shape != (B, Hkv, N, d) or Hkv < 1 or H % Hkv or Nq > N:
         raise ValueError(f"bad shapes {qa.shape} {ka.shape} {va.shape}")
     kvp = None
     if kv_len is not None:
@@ -128,27 +133,26 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
         if kvl.shape != (B,):
             raise ValueError("kv_len must have shape [B]")
         kvp = kvl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
-    R = N if rows is None else len(rows)
+    R = Nq if rows is None else len(rows)
     o = np.zeros((B, H, R, d), dtype=np.float64)
     lse = np.zeros((B, H, R), dtype=np.float64)
     dp = ctypes.POINTER(ctypes.c_double)
-    if qb16:
-        rp = None
-        if rows is not None:
-            ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
-            rp = ra.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
-        u16p = ctypes.POINTER(ctypes.c_uint16)
-        rc = lib.oracle_attn_gqa_bf16(qa.ctypes.data_as(u16p), ka.ctypes.data_as(u16p),
-                                      va.ctypes.data_as(u16p), o.ctypes.data_as(dp),
-                                      lse.ctypes.data_as(dp), B, H, Hkv, N, d, float(scale),
-                                      int(bool(causal)), kvp, rp, R, int(nthreads))
-    else:
-        if rows is not None:
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    rp = None
+    if rows is not None:
+        if not qb16:
             raise ValueError("row subsets are supported for bf16 inputs only")
-        rc = lib.oracle_attn_gqa_f64(qa.ctypes.data_as(dp), ka.ctypes.data_as(dp),
-                                     va.ctypes.data_as(dp), o.ctypes.data_as(dp),
-                                     lse.ctypes.data_as(dp), B, H, Hkv, N, d, float(scale),
-                                     int(bool(causal)), kvp, int(nthreads))
+        ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        rp = ra.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    if qb16:
+        ptrs = (None, None, None, qa.ctypes.data_as(u16p), ka.ctypes.data_as(u16p),
+                va.ctypes.data_as(u16p))
+    else:
+        ptrs = (qa.ctypes.data_as(dp), ka.ctypes.data_as(dp), va.ctypes.data_as(dp),
+                None, None, None)
+    rc = lib.oracle_attn_general(*ptrs, o.ctypes.data_as(dp), lse.ctypes.data_as(dp), B, H,
+                                 Hkv, Nq, N, d, float(scale), int(bool(causal)), kvp, rp, R,
+                                 int(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle returned error {rc}")
     return o, lse

@@ -20,11 +20,16 @@
  * have Hkv <= H heads, H a multiple of Hkv; query head h attends with K/V head
  * h / (H / Hkv). Hkv == H is ordinary multi-head attention.
  *
+ * Fewer queries than keys (Nq <= Nk: the decode / key-value-cache case of
+ * "FlashAttention (UR)", section "Specialised solutions"): query row i stands
+ * at position i + (Nk - Nq) of the key sequence, so with Nq == Nk the mask is
+ * the square one.
+ *
  * Readings taken where the pages are silent:
  *   - scale is passed by the caller (1/sqrt(d) in every workload);
- *   - the mask is additive -inf; causal means key j is allowed iff j <= i
- *     (square, N_q == N_k); key padding masks keys j >= kv_len[b], and query
- *     rows beyond kv_len[b] are still computed against the valid keys;
+ *   - the mask is additive -inf; causal means key j is allowed iff
+ *     j <= i + (Nk - Nq) (square when Nq == Nk); key padding masks keys
+ *     j >= kv_len[b], and query rows are still computed against the valid keys;
  *   - a row with no allowed key gets O = 0 and lse = -inf;
  *   - lse_i = ln sum_j exp(s_ij), natural log, scale included.
  *
@@ -51,11 +56,11 @@ static double bf16_to_f64(uint16_t bits)
     return (double)f;
 }
 
-/* Is key j visible to query row i? */
-static int key_allowed(int i, int j, int causal, int kv_lim)
+/* Is key j visible to query row i (which stands at key position i + off)? */
+static int key_allowed(int i, int j, int causal, int kv_lim, int off)
 {
     if (j >= kv_lim) return 0;
-    if (causal && j > i) return 0;
+    if (causal && j > i + off) return 0;
     return 1;
 }
 
@@ -65,11 +70,11 @@ static int key_allowed(int i, int j, int causal, int kv_lim)
  */
 static void attn_one_row(const double *qi, const double *K, const double *V,
                          int N, int d, double scale, int i, int causal,
-                         int kv_lim, double *srow, double *oi, double *lse_i)
+                         int kv_lim, int off, double *srow, double *oi, double *lse_i)
 {
-    /* s_ij = scale * <q_i, k_j> + mask_ij */
+    /* s_ij = scale * <q_i, k_j> + mask_ij, over the N keys */
     for (int j = 0; j < N; ++j) {
-        if (!key_allowed(i, j, causal, kv_lim)) {
+        if (!key_allowed(i, j, causal, kv_lim, off)) {
             srow[j] = -INFINITY;
             continue;
         }
@@ -118,28 +123,31 @@ static int check_args(int B, int H, int N, int d, double scale, int causal)
  */
 static int attn_driver(const double *qd, const double *kd, const double *vd,
                        const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
-                       double *o, double *lse, int B, int H, int Hkv, int N, int d,
+                       double *o, double *lse, int B, int H, int Hkv, int Nq, int N, int d,
                        double scale, int causal, const int32_t *kv_len,
                        const int32_t *rows, int nrows, int nthreads)
 {
     int rc = check_args(B, H, N, d, scale, causal);
     if (rc) return rc;
+    if (Nq < 0 || Nq > N) return ORACLE_EINVAL;
     if (B == 0 || H == 0) return ORACLE_OK;
     if (Hkv <= 0 || Hkv > H || H % Hkv != 0) return ORACLE_EINVAL;
-    if (nrows < 0 || (rows == NULL && nrows != N)) return ORACLE_EINVAL;
+    if (nrows < 0 || (rows == NULL && nrows != Nq)) return ORACLE_EINVAL;
     if (rows)
         for (int r = 0; r < nrows; ++r)
-            if (rows[r] < 0 || rows[r] >= N) return ORACLE_EINVAL;
+            if (rows[r] < 0 || rows[r] >= Nq) return ORACLE_EINVAL;
     if (B == 0 || H == 0 || nrows == 0) return ORACLE_OK;
     if (N == 0) return ORACLE_EINVAL; /* rows must index into N */
 
-    const size_t head = (size_t)N * d;
+    const size_t head = (size_t)N * d;      /* one K or V head */
+    const size_t qhead = (size_t)Nq * d;    /* one Q head */
+    const int off = N - Nq;                 /* key position of query row 0 */
     const int widen = (qb != NULL);
     double *Kh = NULL, *Vh = NULL, *Qh = NULL;
     if (widen) {
         Kh = (double *)malloc(head * sizeof(double));
         Vh = (double *)malloc(head * sizeof(double));
-        Qh = (double *)malloc(head * sizeof(double));
+        Qh = (double *)malloc((qhead ? qhead : 1) * sizeof(double));
         if (!Kh || !Vh || !Qh) {
             free(Kh); free(Vh); free(Qh);
             return ORACLE_ENOMEM;
@@ -159,12 +167,12 @@ static int attn_driver(const double *qd, const double *kd, const double *vd,
             if (kv_lim > N) kv_lim = N;
         }
         for (int h = 0; h < H; ++h) {
-            const size_t base = ((size_t)b * H + h) * head;                  /* Q, O */
+            const size_t base = ((size_t)b * H + h) * qhead;                 /* Q */
             const size_t kvbase = ((size_t)b * Hkv + h / (H / Hkv)) * head;  /* K, V */
             const double *Q, *K, *V;
             if (widen) {
+                for (size_t e = 0; e < qhead; ++e) Qh[e] = bf16_to_f64(qb[base + e]);
                 for (size_t e = 0; e < head; ++e) {
-                    Qh[e] = bf16_to_f64(qb[base + e]);
                     Kh[e] = bf16_to_f64(kb[kvbase + e]);
                     Vh[e] = bf16_to_f64(vb[kvbase + e]);
                 }
@@ -185,7 +193,7 @@ static int attn_driver(const double *qd, const double *kd, const double *vd,
                     for (int r = 0; r < nrows; ++r) {
                         int i = rows ? rows[r] : r;
                         attn_one_row(Q + (size_t)i * d, K, V, N, d, scale, i,
-                                     causal, kv_lim, srow,
+                                     causal, kv_lim, off, srow,
                                      o_bh + (size_t)r * d, l_bh + r);
                     }
                     free(srow);
@@ -204,7 +212,7 @@ int oracle_attn_f64(const double *q, const double *k, const double *v,
                     int nthreads)
 {
     if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, H, N, d, scale,
+    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, H, N, N, d, scale,
                        causal, kv_len, NULL, N, nthreads);
 }
 
@@ -215,7 +223,7 @@ int oracle_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *rows, int nrows, int nthreads)
 {
     if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, H, N, d, scale,
+    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, H, N, N, d, scale,
                        causal, kv_len, rows, nrows, nthreads);
 }
 
@@ -225,7 +233,7 @@ int oracle_attn_gqa_f64(const double *q, const double *k, const double *v,
                         double scale, int causal, const int32_t *kv_len, int nthreads)
 {
     if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, Hkv, N, d, scale,
+    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, Hkv, N, N, d, scale,
                        causal, kv_len, NULL, N, nthreads);
 }
 
@@ -235,7 +243,22 @@ int oracle_attn_gqa_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          const int32_t *rows, int nrows, int nthreads)
 {
     if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, Hkv, N, d, scale,
+    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, Hkv, N, N, d, scale,
+                       causal, kv_len, rows, nrows, nthreads);
+}
+
+/* General form: q, o [B,H,Nq,d]; k, v [B,Hkv,Nk,d], Nq <= Nk (query row i at
+ * key position i + Nk - Nq). Either fp64 inputs (qd/kd/vd) or bf16 bits
+ * (qb/kb/vb); rows (nullable) as in oracle_attn_bf16, indices into Nq. */
+int oracle_attn_general(const double *qd, const double *kd, const double *vd,
+                        const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
+                        double *o, double *lse, int B, int H, int Hkv, int Nq, int Nk,
+                        int d, double scale, int causal, const int32_t *kv_len,
+                        const int32_t *rows, int nrows, int nthreads)
+{
+    const int fp64 = qd && kd && vd, bits = qb && kb && vb;
+    if (fp64 == bits || !o || !lse) return ORACLE_EINVAL;
+    return attn_driver(qd, kd, vd, qb, kb, vb, o, lse, B, H, Hkv, Nq, Nk, d, scale,
                        causal, kv_len, rows, nrows, nthreads);
 }
 

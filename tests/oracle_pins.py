@@ -243,6 +243,28 @@ def pin_grouped_heads_equal_repeated_heads(lib):
                 assert np.allclose(o3, o[:, perm], atol=TOL, rtol=0)
 
 
+def pin_fewer_queries_are_the_last_rows(lib):
+    """With Nq < Nk queries (query row i standing at key position i + Nk - Nq),
+    each output row equals the matching row of full self-attention over the
+    Nk positions whose last Nq queries are these (the mask and the keys seen
+    are the same)."""
+    rng = np.random.default_rng(21)
+    B, H, Nk, d = 2, 3, 41, 8
+    q_full = rng.standard_normal((B, H, Nk, d))
+    k = rng.standard_normal((B, 1, Nk, d))
+    v = rng.standard_normal((B, 1, Nk, d))
+    for Nq in (1, 5, 41):
+        for causal, kvl in [(True, None), (False, None), (True, [41, 30]), (False, [12, 41])]:
+            o_full, l_full = _attn(lib, q_full, k, v, 0.45, causal, kvl)
+            o, lse = _attn(lib, q_full[:, :, Nk - Nq:], k, v, 0.45, causal, kvl)
+            assert np.array_equal(o, o_full[:, :, Nk - Nq:]), (Nq, causal, kvl)
+            assert np.array_equal(lse, l_full[:, :, Nk - Nq:]), (Nq, causal, kvl)
+    # a single causal query at the last position sees every key: the non-causal answer
+    o1, _ = _attn(lib, q_full[:, :, -1:], k, v, 0.45, True)
+    o2, _ = _attn(lib, q_full[:, :, -1:], k, v, 0.45, False)
+    assert np.array_equal(o1, o2)
+
+
 ALL_PINS = [
     pin_golden_closed_forms,
     pin_rows_sum_to_one,
@@ -255,6 +277,7 @@ ALL_PINS = [
     pin_online_equals_full,
     pin_no_visible_key,
     pin_grouped_heads_equal_repeated_heads,
+    pin_fewer_queries_are_the_last_rows,
 ]
 
 

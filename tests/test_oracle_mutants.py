@@ -17,10 +17,12 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_ref.c")
 
 MUTANTS = {
     "dropped_scale": ("srow[j] = scale * dot;", "srow[j] = dot;"),
-    "causal_direction_flipped": ("if (causal && j > i) return 0;",
-                                 "if (causal && j < i) return 0;"),
-    "causal_diagonal_hidden": ("if (causal && j > i) return 0;",
-                               "if (causal && j >= i) return 0;"),
+    "causal_direction_flipped": ("if (causal && j > i + off) return 0;",
+                                 "if (causal && j < i + off) return 0;"),
+    "causal_diagonal_hidden": ("if (causal && j > i + off) return 0;",
+                               "if (causal && j >= i + off) return 0;"),
+    "causal_offset_dropped": ("if (causal && j > i + off) return 0;",
+                              "if (causal && j > i) return 0;"),
     "kv_len_off_by_one": ("if (j >= kv_lim) return 0;", "if (j > kv_lim) return 0;"),
     "lse_log2": ("double lse = m + log(sum);", "double lse = m + log2(sum);"),
     "lse_missing_max": ("double lse = m + log(sum);", "double lse = log(sum);"),
