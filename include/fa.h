@@ -22,7 +22,7 @@
  *   - q, k, v, o must be 16-byte aligned (the tensor-memory-access engine
  *     requires it); lse 4-byte aligned. o and lse must not overlap each other
  *     or the inputs.
- *   - d must be 64 or 128; anything else returns FA_ERR_UNSUPPORTED.
+ *   - d must be 64, 128 or 256; anything else returns FA_ERR_UNSUPPORTED.
  *   - B, H, N >= 0. If any is 0 there is nothing to compute: the call returns
  *     FA_OK without launching (pointers may then be NULL).
  *   - scale must be finite and > 0; causal must be 0 or 1.
@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARG = 1,  /* null/misaligned/overlapping pointer, bad size, scale, causal */
-    FA_ERR_UNSUPPORTED = 2,  /* head dim other than 64/128, or not an sm_100 device */
+    FA_ERR_UNSUPPORTED = 2,  /* head dim other than 64/128/256, or not an sm_100 device */
     FA_ERR_LAUNCH = 3,       /* the CUDA runtime refused the launch or a sync failed */
     FA_ERR_TIMEOUT = 4       /* a kernel's bounded wait ran out (see fa_last_device_error) */
 } fa_status_t;

@@ -48,7 +48,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 struct DeviceState {
     bool probed = false;
     bool supported = false;
-    bool smem_set[2] = {false, false};  // d = 64, 128
+    bool smem_set[3] = {false, false, false};  // d = 64, 128, 256
     uint32_t* err_ptr = nullptr;
 };
 
@@ -90,13 +90,18 @@ int prepare_device(int d, int* dev_out, uint32_t** err_out) {
         st.probed = true;
     }
     if (!st.supported) return FA_ERR_UNSUPPORTED;
-    const int di = (d == 128) ? 1 : 0;
+    const int di = (d == 256) ? 2 : (d == 128) ? 1 : 0;
     if (!st.smem_set[di]) {
-        cudaError_t e = (d == 128)
-            ? cudaFuncSetAttribute(fa_fwd_sm100<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   Cfg<128>::kSmemBytes)
-            : cudaFuncSetAttribute(fa_fwd_sm100<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   Cfg<64>::kSmemBytes);
+        cudaError_t e =
+            (d == 256) ? cudaFuncSetAttribute(fa_fwd_sm100<256>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              Cfg<256>::kSmemBytes)
+            : (d == 128) ? cudaFuncSetAttribute(fa_fwd_sm100<128>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128>::kSmemBytes)
+                         : cudaFuncSetAttribute(fa_fwd_sm100<64>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64>::kSmemBytes);
         if (e != cudaSuccess) return FA_ERR_LAUNCH;
         st.smem_set[di] = true;
     }
@@ -135,7 +140,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (B == 0 || H == 0 || N == 0) return FA_OK;
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     const uintptr_t a16 = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -145,8 +150,9 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     if ((reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0) return FA_ERR_INVALID_ARG;
     const int64_t BH = (int64_t)B * H;
     const int64_t BHkv = (int64_t)B * H_kv;
-    const int64_t n_pairs = ((int64_t)N + 255) / 256;
-    if (BH > INT32_MAX || BH * n_pairs > INT32_MAX) return FA_ERR_INVALID_ARG;
+    const int64_t rows_per_unit = (d == 256) ? 128 : 256;   // query tiles per unit x 128
+    const int64_t n_units = ((int64_t)N + rows_per_unit - 1) / rows_per_unit;
+    if (BH > INT32_MAX || BH * n_units > INT32_MAX) return FA_ERR_INVALID_ARG;
     const size_t elems = (size_t)BH * (size_t)N * (size_t)d;
     if ((double)BH * N * d > 9.0e18) return FA_ERR_INVALID_ARG;
     const size_t tbytes = elems * 2, lbytes = (size_t)BH * (size_t)N * 4;
@@ -176,7 +182,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.H = H;
     p.H_kv = H_kv;
     p.N = N;
-    p.n_pairs = (int)n_pairs;
+    p.n_units = (int)n_units;
     // Launch-order head groups: as few groups as keep a group's K/V (2*N*d*2
     // bytes per K/V head, shared by H / H_kv query heads) within
     // kL2GroupBytes, with the query heads split evenly.
@@ -188,9 +194,11 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.scale_log2 = scale * 1.4426950408889634f;
     p.watchdog_ns = kWatchdogNs;
 
-    const dim3 grid((unsigned)(BH * n_pairs)), block(kThreads);
+    const dim3 grid((unsigned)(BH * n_units)), block(kThreads);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 128)
+    if (d == 256)
+        fa_fwd_sm100<256><<<grid, block, Cfg<256>::kSmemBytes, s>>>(mq, mk, mv, p);
+    else if (d == 128)
         fa_fwd_sm100<128><<<grid, block, Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
     else
         fa_fwd_sm100<64><<<grid, block, Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);

@@ -62,6 +62,8 @@
 // and p_full phases, where n_t is the tile's number of key tiles (an idle
 // tile still takes part in its once-per-unit hand-offs), so every role can
 // compute every phase index and no barrier runs two phases ahead of a waiter.
+// (With one query tile the epilogue may find o_done two phases short of the
+// unit's last, so it waits for the last two phases in turn.)
 #pragma once
 
 #include <cuda_bf16.h>
@@ -78,18 +80,29 @@ constexpr int kTmaWarp = 9;
 constexpr float kMaxTileSum = 18446744073709551616.0f;  // 2^64
 constexpr float kLn2 = 0.69314718055994530942f;
 
+// Per head dimension. d = 64, 128: a unit is two query tiles, each with one
+// S buffer (TMEM: S0 | S1 | O0 | O1). d = 256: O alone takes 256 TMEM columns,
+// so a unit is one query tile whose S is double-buffered (TMEM: Sa | Sb | O):
+// the tensor cores compute the next tile's scores while the softmax works on
+// the current ones, and at d = 256 each key tile carries twice the MMA work.
 template <int D>
 struct Cfg {
-    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static_assert(D == 64 || D == 128 || D == 256, "head dim 64, 128 or 256");
+    static constexpr int kQT = (D == 256) ? 1 : 2;        // query tiles per unit
     static constexpr int kBlocks = D / 64;                // 128-byte column blocks per row
     static constexpr int kBlockBytes = kTile * 128;       // 16 KB
     static constexpr int kTileBytes = kTile * D * 2;      // one Q/K/V tile
-    static constexpr int kSlots = (D == 128) ? 4 : 8;     // K/V ring depth
-    static constexpr int kSmemTiles = (2 + kSlots) * kTileBytes;
+    static constexpr int kSlots = (D == 256) ? 2 : (D == 128) ? 4 : 8;  // K/V ring depth
+    static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 1024 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
-    __device__ static constexpr uint32_t col_s(int t) { return (uint32_t)(t * 128); }
+    static constexpr int kUnitConsumers = 1 + 4 * kQT;   // MMA thread + one lane per softmax warp
+    // S buffer b (a query tile's, or with one tile the buffer of key-tile parity b)
+    __device__ static constexpr uint32_t col_s(int b) { return (uint32_t)(b * 128); }
     __device__ static constexpr uint32_t col_o(int t) { return 256u + (uint32_t)(t * D); }
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static_assert(kSlots <= 8, "K/V ring barriers");
+    static_assert(256 + kQT * D <= (int)kTmemCols, "TMEM columns");
 };
 
 struct FwdParams {
@@ -99,7 +112,7 @@ struct FwdParams {
     uint32_t* dev_err;         // status word
     int B, H, N;
     int H_kv;                  // K/V heads; query head h reads K/V head h / (H / H_kv)
-    int n_pairs;               // ceil(N / 256)
+    int n_units;               // units per head: ceil(N / (128 * query tiles per unit))
     int group_heads;           // heads per L2 group (launch order)
     int causal;
     float scale_log2;          // scale * log2(e)
@@ -127,7 +140,6 @@ struct SmemBarriers {
 };
 static_assert(sizeof(SmemBarriers) <= 1024, "barrier region");
 static_assert(offsetof(SmemBarriers, clc_resp) % 16 == 0, "CLC response alignment");
-constexpr int kUnitConsumers = 1 + 8;  // MMA thread + one lane per softmax warp
 
 // One work unit, decoded from its launch-order index.
 struct Unit {
@@ -145,22 +157,23 @@ __device__ __forceinline__ int kv_tiles_for(int q_first, int N, int kv_lim, int 
     return (lim + kTile - 1) / kTile;
 }
 
+template <int QT>
 __device__ __forceinline__ Unit decode_unit(int id, const FwdParams& p) {
     Unit u;
     const int BH = p.B * p.H;
-    const int per_group = p.group_heads * p.n_pairs;
+    const int per_group = p.group_heads * p.n_units;
     const int grp = id / per_group;
     const int in_grp = id - grp * per_group;
     const int heads_here = min(p.group_heads, BH - grp * p.group_heads);
-    const int pair = p.n_pairs - 1 - in_grp / heads_here;
+    const int pair = p.n_units - 1 - in_grp / heads_here;
     u.bh = grp * p.group_heads + in_grp % heads_here;
     u.b = u.bh / p.H;
     u.bkv = u.b * p.H_kv + (u.bh - u.b * p.H) / (p.H / p.H_kv);
-    u.q0 = pair * 2 * kTile;
+    u.q0 = pair * QT * kTile;
     u.kv_lim = p.N;
     if (p.kv_len != nullptr) u.kv_lim = max(0, min(p.N, p.kv_len[u.b]));
     u.n[0] = kv_tiles_for(u.q0, p.N, u.kv_lim, p.causal);
-    u.n[1] = kv_tiles_for(u.q0 + kTile, p.N, u.kv_lim, p.causal);
+    u.n[1] = (QT == 2) ? kv_tiles_for(u.q0 + kTile, p.N, u.kv_lim, p.causal) : 0;
     u.n_max = max(u.n[0], u.n[1]);
     return u;
 }
@@ -207,8 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ[2] = {smem, smem + C::kTileBytes};
-    uint8_t* sKV = smem + 2 * C::kTileBytes;
+    // Q tiles (kQT of them), then the K/V ring, then the barriers.
+    uint8_t* sQ[2] = {smem, smem + C::kTileBytes};   // sQ[1] is used only when kQT == 2
+    uint8_t* sKV = smem + C::kQT * C::kTileBytes;
     SmemBarriers* bars = reinterpret_cast<SmemBarriers*>(smem + C::kSmemTiles);
 
     const int tid = threadIdx.x;
@@ -225,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->o_done[t], 1);
             mbar_init(&bars->o_empty[t], kTile);
             mbar_init(&bars->unit_full[t], 1);
-            mbar_init(&bars->unit_empty[t], kUnitConsumers);
+            mbar_init(&bars->unit_empty[t], C::kUnitConsumers);
             mbar_init(&bars->clc_bar[t], 1);
         }
         mbar_init(&bars->teardown, 1);
@@ -265,16 +279,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t clc_pending_parity = 0;
             int q_unit[2] = {-1, -1};  // last unit whose Q tile t was requested
             bool ok = true;
-            auto load_kv = [&](const Unit& u, int jj) -> bool {   // jj-th K/V load of unit u
+            // jj-th K/V load of unit u, in the order the MMAs consume them:
+            // two query tiles: K0 V0 K1 V1 ...; one query tile (S double-
+            // buffered): K0 K1 V0 K2 V1 K3 V2 ... V(n-2) V(n-1).
+            auto load_kv = [&](const Unit& u, int jj) -> bool {
+                bool is_v;
+                int tile;
+                if (C::kQT == 2) {
+                    is_v = (jj & 1) != 0;
+                    tile = jj >> 1;
+                } else {
+                    const int n = u.n[0];
+                    const int kfirst = min(2, n);
+                    const int paired = 2 * max(0, n - 2);
+                    const int q = jj - kfirst;
+                    if (q < 0) {
+                        is_v = false;
+                        tile = jj;
+                    } else if (q < paired) {
+                        is_v = (q & 1) == 0;
+                        tile = is_v ? q / 2 : q / 2 + 2;
+                    } else {
+                        is_v = true;
+                        tile = max(0, n - 2) + (q - paired);
+                    }
+                }
                 const int slot = L % C::kSlots;
                 const uint32_t round = (uint32_t)(L / C::kSlots);
                 if (!mbar_wait(&bars->kv_empty[slot], (round & 1u) ^ 1u, wd)) return false;
-                const CUtensorMap* map = (jj & 1) ? &tm_v : &tm_k;
+                const CUtensorMap* map = is_v ? &tm_v : &tm_k;
                 uint8_t* dst = sKV + slot * C::kTileBytes;
                 mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
                 for (int blk = 0; blk < C::kBlocks; ++blk)
                     tma_load_3d_hint(map, &bars->kv_full[slot], dst + blk * C::kBlockBytes,
-                                     blk * 64, (jj >> 1) * kTile, u.bkv, pol_kv);
+                                     blk * 64, tile * kTile, u.bkv, pol_kv);
                 ++L;
                 return true;
             };
@@ -285,13 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bars->unit_id[us] = id;
                 mbar_arrive(&bars->unit_full[us]);
                 if (id < 0) break;
-                const Unit u = decode_unit(id, p);
-                // K_0 and V_0 first: the ring has room while the previous unit's
-                // last tiles are consumed, and Q may have to wait for it.
+                const Unit u = decode_unit<C::kQT>(id, p);
+                // The first two K/V loads go first: the ring has room while the
+                // previous unit's last tiles are consumed, and Q may have to wait.
                 const int early = min(2, 2 * u.n_max);
                 for (int jj = 0; ok && jj < early; ++jj) ok = load_kv(u, jj);
                 // Q tiles (one q_full phase per unit and tile, possibly with no bytes)
-                for (int t = 0; t < 2 && ok; ++t) {
+                for (int t = 0; t < C::kQT && ok; ++t) {
                     if (k > 0) ok = mbar_wait(&bars->q_empty[t], (uint32_t)((k - 1) & 1), wd);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bars->q_full[t], u.n[t] > 0 ? C::kTileBytes : 0);
@@ -323,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int l2 = max(0, L - C::kSlots); l2 < L; ++l2)
                 mbar_wait_drain(&bars->kv_full[l2 % C::kSlots], (uint32_t)(l2 / C::kSlots) & 1u,
                                 wd);
-            for (int t = 0; t < 2; ++t)
+            for (int t = 0; t < C::kQT; ++t)
                 if (q_unit[t] >= 0) mbar_wait_drain(&bars->q_full[t], (uint32_t)(q_unit[t] & 1), wd);
         }
         __syncwarp();
@@ -331,35 +369,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ====================================================== MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTile, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+            constexpr int kPvN = (D > 128) ? 128 : D;          // N of one P.V MMA
+            constexpr int kPvHalves = D / kPvN;
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kPvN, 0, 1);
             // Descriptors are built once; a tile's start address is added in
             // 16-byte units to the low field (addresses stay below 256 KB).
             const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ[0]), 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(smem_u32(sKV), 16, 1024);            // K-major
             const uint64_t dv0 = smem_desc_sw128(smem_u32(sKV), C::kBlockBytes, 1024); // MN-major
             constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
-            auto issue_qk = [&](int t, int slot) {
+            // S buffer sb = Q tile t . K tile in `slot`
+            auto issue_qk = [&](int t, int sb, int slot) {
                 const uint64_t a = dq0 + (uint64_t)t * kTileStep;
                 const uint64_t b = dk0 + (uint64_t)slot * kTileStep;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t off =
                         (uint64_t)(((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4);
-                    umma_ss(tmem + C::col_s(t), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + C::col_s(sb), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int t, int slot, bool accumulate) {
+            // O of tile t (+)= P in S buffer sb . V tile in `slot`. At d = 256 each
+            // K-step is issued as two N = 128 MMAs, one per half of V's column
+            // blocks (the same instruction shape as d = 128).
+            auto issue_pv = [&](int t, int sb, int slot, bool accumulate) {
                 const uint64_t b = dv0 + (uint64_t)slot * kTileStep;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
-                    umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + (uint32_t)(kk * 8),
-                            b + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
-                            (accumulate || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int h = 0; h < kPvHalves; ++h) {
+                        umma_ts(tmem + C::col_o(t) + (uint32_t)(h * kPvN),
+                                tmem + C::col_s(sb) + (uint32_t)(kk * 8),
+                                b + (uint64_t)((kk * 16 * 128 + h * (kPvN / 64) * C::kBlockBytes) >> 4),
+                                idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                    }
                 }
             };
             bool ok = true;
             int L0 = 0;                         // index of this unit's first K/V load
             uint32_t ph_p[2] = {0u, 0u};        // p_full phases consumed
+            if constexpr (C::kQT == 2) {
             for (int k = 0; ok; ++k) {
                 const int us = k & 1;
                 ok = mbar_wait(&bars->unit_full[us], (uint32_t)((k >> 1) & 1), wd);
@@ -367,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int id = bars->unit_id[us];
                 mbar_arrive(&bars->unit_empty[us]);
                 if (id < 0) break;
-                const Unit u = decode_unit(id, p);
+                const Unit u = decode_unit<C::kQT>(id, p);
                 // O_t is free once the previous unit's epilogue has read it
                 bool o_ready[2] = {k == 0, k == 0};
                 for (int t = 0; t < 2 && ok; ++t)
@@ -379,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         for (int t = 0; t < 2; ++t) {
                             if (u.n[t] > 0) {
-                                issue_qk(t, L0 % C::kSlots);
+                                issue_qk(t, t, L0 % C::kSlots);
                                 umma_commit(&bars->s_full[t]);
                                 if (u.n[t] == 1) umma_commit(&bars->q_empty[t]);  // last Q.K^T
                             }
@@ -403,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (!ok) break;
                         tc_fence_after();
-                        issue_pv(t, sV, j > 0);
+                        issue_pv(t, t, sV, j > 0);
                         umma_commit(&bars->o_done[t]);
                         if (j + 1 < u.n[t]) {
                             if (!k_ready) {
@@ -413,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tc_fence_after();
                                 k_ready = true;
                             }
-                            issue_qk(t, sK);
+                            issue_qk(t, t, sK);
                             umma_commit(&bars->s_full[t]);
                             if (j + 2 == u.n[t]) umma_commit(&bars->q_empty[t]);  // last Q.K^T
                         }
@@ -433,20 +482,85 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 L0 += 2 * u.n_max;
             }
+            } else {
+            // One query tile, S double-buffered: QK(0) QK(1) | PV(0) QK(2) | PV(1) QK(3) ...
+            // QK(j+2) overwrites the buffer PV(j) reads, after it in issue order.
+            for (int k = 0; ok; ++k) {
+                const int us = k & 1;
+                ok = mbar_wait(&bars->unit_full[us], (uint32_t)((k >> 1) & 1), wd);
+                if (!ok) break;
+                const int id = bars->unit_id[us];
+                mbar_arrive(&bars->unit_empty[us]);
+                if (id < 0) break;
+                const Unit u = decode_unit<C::kQT>(id, p);
+                const int n = u.n[0];
+                bool o_ready = (k == 0);
+                // positions of K_t and V_j in this unit's load order (see the producer)
+                auto posK = [&](int t) { return t < 2 ? t : 2 * t - 1; };
+                auto posV = [&](int j) { return (j <= n - 3) ? 2 + 2 * j : n + j; };
+                auto slot_of = [&](int pos) { return (L0 + pos) % C::kSlots; };
+                auto wait_load = [&](int pos) -> bool {
+                    const int L = L0 + pos;
+                    return mbar_wait(&bars->kv_full[L % C::kSlots],
+                                     (uint32_t)(L / C::kSlots) & 1u, wd);
+                };
+                ok = mbar_wait(&bars->q_full[0], (uint32_t)(k & 1), wd);
+                for (int t = 0; ok && t < min(2, n); ++t) {
+                    ok = wait_load(posK(t));
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(0, t, slot_of(posK(t)));
+                    umma_commit(&bars->s_full[t]);
+                    umma_commit(&bars->kv_empty[slot_of(posK(t))]);
+                    if (t == n - 1) umma_commit(&bars->q_empty[0]);   // last Q.K^T
+                }
+                for (int j = 0; ok && j < n; ++j) {
+                    const int b = j & 1;
+                    ok = wait_load(posV(j));
+                    if (!ok) break;
+                    ok = mbar_wait(&bars->p_full[b], ph_p[b] & 1u, wd);
+                    ++ph_p[b];
+                    if (ok && !o_ready) {
+                        ok = mbar_wait(&bars->o_empty[0], (uint32_t)((k - 1) & 1), wd);
+                        o_ready = true;
+                    }
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(0, b, slot_of(posV(j)), j > 0);
+                    umma_commit(&bars->o_done[0]);
+                    umma_commit(&bars->kv_empty[slot_of(posV(j))]);
+                    if (j + 2 < n) {
+                        ok = wait_load(posK(j + 2));
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_qk(0, b, slot_of(posK(j + 2)));
+                        umma_commit(&bars->s_full[b]);
+                        umma_commit(&bars->kv_empty[slot_of(posK(j + 2))]);
+                        if (j + 2 == n - 1) umma_commit(&bars->q_empty[0]);   // last Q.K^T
+                    }
+                }
+                if (!ok) break;
+                if (n == 0) {                          // idle unit: its once-per-unit hand-offs
+                    umma_commit(&bars->q_empty[0]);
+                    if (!o_ready) ok = mbar_wait(&bars->o_empty[0], (uint32_t)((k - 1) & 1), wd);
+                    umma_commit(&bars->o_done[0]);
+                }
+                L0 += 2 * n;
+            }
+            }
             // Drain: all MMAs issued by this thread complete before teardown.
             umma_commit(&bars->teardown);
             mbar_wait_drain(&bars->teardown, 0u, wd);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 4 * C::kQT) {
         // ====================================================== softmax warpgroups
         const int t = warp >> 2;                      // query tile 0 or 1
         const int row = tid & (kTile - 1);            // row within the tile == TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + C::col_s(t);
         const uint32_t tO = tmem + lane_base + C::col_o(t);
         const float c = p.scale_log2;
-        uint32_t ph_s = 0;     // s_full phases consumed
+        uint32_t ph_s[2] = {0u, 0u};   // s_full phases consumed (per S buffer)
         uint32_t o_base = 0;   // o_done phases of earlier units
         bool ok = true;
         for (int k = 0; ok; ++k) {
@@ -458,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->unit_empty[us]);
             if (id < 0) break;
-            const Unit u = decode_unit(id, p);
+            const Unit u = decode_unit<C::kQT>(id, p);
             const int n = u.n[t];
             const int i = u.q0 + t * kTile + row;     // global query row
             const int lim_row = p.causal ? min(u.kv_lim, i + 1) : u.kv_lim;  // visible: j < lim_row
@@ -466,8 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             float l = 0.f;             // running sum of exp2((s - m_ref) * c)
 
             for (int j = 0; j < n; ++j) {
-                ok = mbar_wait(&bars->s_full[t], ph_s & 1u, wd);
-                ++ph_s;
+                const int sb = (C::kQT == 2) ? t : (j & 1);   // this tile's S buffer
+                const uint32_t tS = tmem + lane_base + C::col_s(sb);
+                ok = mbar_wait(&bars->s_full[sb], ph_s[sb] & 1u, wd);
+                ++ph_s[sb];
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
@@ -532,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars->p_full[t]);
+                mbar_arrive(&bars->p_full[sb]);
             }
             if (!ok) break;
 
@@ -540,6 +656,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the unit's last o_done phase for this tile (its idle phase if n == 0)
             const uint32_t last = o_base + (uint32_t)(n > 0 ? n - 1 : 0);
             o_base += (uint32_t)(n > 0 ? n : 1);
+            if (C::kQT == 1 && n >= 2) {
+                // With one query tile the last score tile was issued after
+                // P.V(n-3) only, so o_done may still be in phase n-2: a parity
+                // wait for phase n-1 alone would pass at once. Wait in order.
+                ok = mbar_wait(&bars->o_done[t], (last - 1u) & 1u, wd);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
             ok = mbar_wait(&bars->o_done[t], last & 1u, wd);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -547,39 +671,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool write = i < p.N;
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
             __nv_bfloat16* orow = p.o + ((size_t)u.bh * p.N + (size_t)i) * D;
-            uint32_t r[D];
-            if (n > 0) {
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t* rc = r + ch * 32;
-                    tmem_ld32(tO + (uint32_t)(ch * 32), *reinterpret_cast<uint32_t(*)[32]>(rc));
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t r[32];
+                if (n > 0) {
+                    tmem_ld32(tO + (uint32_t)(ch * 32), r);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) r[q] = 0u;
                 }
-                tmem_wait_ld();
-            } else {
+                if (ch == D / 32 - 1) {
+                    // O has been read: the next unit's first P.V may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(&bars->o_empty[t]);
+                }
+                if (write) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-                for (int q = 0; q < D; ++q) r[q] = 0u;
+                    for (int v = 0; v < 4; ++v) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv_l,
+                                          __uint_as_float(r[8 * v + 1]) * inv_l);
+                        w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_l,
+                                          __uint_as_float(r[8 * v + 3]) * inv_l);
+                        w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_l,
+                                          __uint_as_float(r[8 * v + 5]) * inv_l);
+                        w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_l,
+                                          __uint_as_float(r[8 * v + 7]) * inv_l);
+                        dst[v] = w;
+                    }
+                }
             }
-            // O has been read: the next unit's first P.V may overwrite it
-            tc_fence_before();
-            mbar_arrive(&bars->o_empty[t]);
-            if (write) {
-                uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-                for (int v = 0; v < D / 8; ++v) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv_l,
-                                      __uint_as_float(r[8 * v + 1]) * inv_l);
-                    w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_l,
-                                      __uint_as_float(r[8 * v + 3]) * inv_l);
-                    w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_l,
-                                      __uint_as_float(r[8 * v + 5]) * inv_l);
-                    w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_l,
-                                      __uint_as_float(r[8 * v + 7]) * inv_l);
-                    dst[v] = w;
-                }
+            if (write)
                 p.lse[(size_t)u.bh * p.N + (size_t)i] =
                     (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
-            }
         }
     }
 

@@ -63,7 +63,8 @@ def call(lib, **over):
     (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
     (dict(scale=-0.1), fa.FA_ERR_INVALID_ARG),
     (dict(d=96), fa.FA_ERR_UNSUPPORTED),
-    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=192), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=512), fa.FA_ERR_UNSUPPORTED),
     (dict(q=0), fa.FA_ERR_INVALID_ARG),
     (dict(lse=0), fa.FA_ERR_INVALID_ARG),
     (dict(q=P + 8), fa.FA_ERR_INVALID_ARG),          # not 16-byte aligned

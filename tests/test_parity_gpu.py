@@ -105,7 +105,7 @@ def test_workload_sampled_rows(fa, idx):
 RAGGED = [1, 17, 127, 128, 129, 255, 256, 257, 300, 383, 513]
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", RAGGED)
 def test_ragged_lengths(fa, N, causal, d):
@@ -113,7 +113,7 @@ def test_ragged_lengths(fa, N, causal, d):
     check_full(fa, q, k, v, causal, what=f"N={N} causal={causal} d={d}")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_key_padding_edges(fa, causal, d):
     N = 300
@@ -142,8 +142,28 @@ def test_persistent_many_heads_d128(fa):
     check_full(fa, q, k, v, True, what="persistent 300 heads d=128")
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_dim_256_long(fa, causal):
+    """d = 256 (one query tile per unit, double-buffered scores) over many key
+    tiles and units, with mixed key-padding lengths."""
+    B, H, N, d = 4, 12, 1100, 256
+    q, k, v, _ = workloads.make_custom(B, H, N, d, seed=256 + causal)
+    kv_len = torch.tensor([1100, 700, 1, 0], dtype=torch.int32)
+    check_full(fa, q, k, v, causal, kv_len, what=f"d=256 causal={causal}")
+
+
+def test_head_dim_256_sampled_full_size(fa):
+    """Long sequence at d = 256: sampled rows against the oracle."""
+    B, H, N, d = 1, 4, 8192, 256
+    q, k, v, _ = workloads.make_custom(B, H, N, d, seed=2560)
+    o, lse = run_gpu(fa, q, k, v, True)
+    rows = workloads.sample_rows(N, seed=7, n_random=48, edge=48)
+    o_ref, lse_ref = oracle.attention(q, k, v, 1 / math.sqrt(d), causal=True, rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], o_ref, lse_ref, "d=256 N=8192 causal")
+
+
 @pytest.mark.parametrize("H,H_kv", [(8, 2), (6, 1), (4, 4)])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_grouped_and_multi_query(fa, H, H_kv, d, causal):
     """K/V heads shared by groups of query heads (H_kv = 1: multi-query)."""
