@@ -2,7 +2,7 @@
 """Benchmark of the fused attention forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 5]
+                    [--workload 5] [--decode 1]
 
 A step is one full forward (one kernel launch) over the workload's tensors,
 which are resident in device memory before the timed region starts. The
@@ -18,6 +18,9 @@ only a barrier and a max-reduction of the timings ("scaling": "weak").
 --impl reference times the CPU oracle (fp64 C, the machine's host cores) on a
 bounded row sample of the same workload, in the same unit; under torchrun only
 rank 0 runs it.
+
+--decode 1 times the split-KV path instead (one query row per head against an
+8K-key cache with grouped K/V heads), in GB/s of algorithmic bytes.
 """
 from __future__ import annotations
 
@@ -383,7 +386,7 @@ def our_arm(args, w):
                 "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
                 "algorithmic_bytes": float(w.B * w.N * (2 * w.H * w.d * 2 + 2 * w.kv_heads * w.d * 2
                                                         + 4 * w.H)),
-                "kernel": f"fa_fwd_sm100<{w.d}>"}
+                "kernel": f"fa_fwd_sm100<{w.d},{1 if w.d == 256 else 2},square>"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -415,6 +418,151 @@ def our_arm(args, w):
     return 0
 
 
+def decode_arm(args, w):
+    """Split-KV decoding: one fa_fwd_splitkv call per step (the attention
+    kernel over all key ranges, then the log-sum-exp merge) at the library's
+    default number of ranges. Memory-bound: reported in GB/s of algorithmic
+    bytes (K, V and Q read once, O and lse written once) against the measured
+    copy bandwidth. Replicas only under torchrun, like the square arm."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import io_aware_exact_18_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.load_library()
+    q, k, v, _ = workloads.make_qkv(w.B, w.H, w.H_kv, w.Nq, w.Nk, w.d, seed=w.seed + 1000 * rank)
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    od = torch.empty_like(qd)
+    lsed = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    splits = fa.fa_splitkv_default_splits(w.B, w.H, w.H_kv, w.Nq, w.Nk, w.d)
+    ws_bytes = fa.fa_splitkv_workspace_bytes(w.B, w.H, w.Nq, w.d, splits)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+
+    def step():
+        st = fa.fa_fwd_splitkv(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                               lsed.data_ptr(), w.B, w.H, w.H_kv, w.Nq, w.Nk, w.d, w.scale,
+                               int(w.causal), None, splits, ws.data_ptr(), ws_bytes, sh)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_fwd_splitkv")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    st = fa.fa_last_device_error(sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed region")
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    nbytes = w.algorithmic_bytes()
+    value = world * nbytes / (ms * 1e-3) / 1e9
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    # end to end: the step's inputs (q and the K/V cache) copied from pinned
+    # host memory, the call, O and lse read back
+    e2e_steps = max(1, min(args.steps, 5))
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    lh = torch.empty(lsed.shape, dtype=lsed.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            fa.decode_attention(qd, kd, vd, scale=w.scale, causal=w.causal, num_splits=splits,
+                                out=od, lse=lsed, workspace=ws, stream=sh)
+            oh.copy_(od, non_blocking=True)
+            lh.copy_(lsed, non_blocking=True)
+
+    e2e_step()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * nbytes / (e2e_ms * 1e-3) / 1e9
+
+    peaks, peak_src = load_peaks()
+    achieved = nbytes / (ms_local * 1e-3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peak_src} copy bandwidth",
+                "algorithmic_bytes": float(nbytes),
+                "timed": "whole step: attention kernel over all key ranges + merge kernel",
+                "kernel": f"fa_fwd_sm100<{w.d},1,general> + fa_splitkv_combine<{w.d}>"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nthreads = os.cpu_count() or 1
+        t = time.perf_counter()
+        oracle.attention(q, k, v, w.scale, causal=w.causal, nthreads=nthreads)
+        dt = time.perf_counter() - t
+        cpu = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+               "sample": f"the whole step ({w.B * w.H} query rows x {w.Nk} keys), fp64, "
+                         f"{nthreads} threads", "seconds": dt}
+    if rank == 0:
+        line = {
+            "metric": "split-KV decode attention GB/s (K, V, Q read once; O, lse written once)",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**w.describe(), "num_splits": splits,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "no flush: the K/V cache ({:.0f} MiB) exceeds the 126 MB L2".format(
+                           2 * w.B * w.H_kv * w.Nk * w.d * 2 / 2**20)},
+            "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps * (2 if splits > 1 else 1),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -428,8 +576,20 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", default=None,
+                    help="time the split-KV decode path on this decode workload "
+                         "(name, or 1 for the first) instead of square attention")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.decode:
+        dw = (workloads.DECODE_WORKLOADS[int(args.decode) - 1] if args.decode.isdigit()
+              else workloads.DECODE_BY_NAME[args.decode])
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the decode line has no reference arm; its cpu_baseline key "
+                              "times the oracle"}), flush=True)
+            return 0
+        return decode_arm(args, dw)
     if args.shape:
         f = [int(x) for x in args.shape.split(",")]
         B, H, N, d = f[:4]

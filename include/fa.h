@@ -41,6 +41,7 @@
 #ifndef FA_H_
 #define FA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -88,6 +89,58 @@ int fa_fwd_kvlen(const void *q, const void *k, const void *v, void *o, float *ls
 int fa_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse,
                int B, int H, int H_kv, int N, int d, float scale, int causal,
                const int32_t *kv_len, void *stream);
+
+/* Largest num_splits fa_fwd_splitkv accepts. */
+#define FA_MAX_SPLITS 128
+
+/*
+ * Split-KV forward for few queries against many keys (decoding with a key-value
+ * cache; the specialised inference kernels of "FlashAttention (UR)", section
+ * "Specialised solutions"). The result is the same attention as above:
+ *   q, o: bf16 [B, H, Nq, d]; lse: fp32 [B, H, Nq];
+ *   k, v: bf16 [B, H_kv, Nk, d], H a multiple of H_kv (grouped heads as in
+ *   fa_fwd_gqa); 0 <= Nq <= Nk.
+ * Query row i stands at key position i + Nk - Nq: with causal = 1 it sees keys
+ * j <= i + Nk - Nq (Nq == Nk is the square mask of fa_fwd). kv_len (nullable)
+ * hides keys j >= kv_len[b] as in fa_fwd_kvlen; the causal offset stays
+ * Nk - Nq.
+ * Each row's keys are cut into num_splits contiguous ranges of whole 128-key
+ * tiles, handled by different CTAs; each range's normalised output and
+ * log-sum-exp go to `workspace`, and a second kernel merges them by
+ * lse-weighted rescaling (the online-softmax update of section "Online
+ * softmax", applied once per range). The query heads that share a K/V head
+ * are processed together, so each K/V tile is read once per group.
+ *   num_splits: 1..FA_MAX_SPLITS (1: no workspace, one kernel; more splits
+ *     than key tiles leave some ranges empty, which is allowed).
+ *   workspace: device memory owned by the caller, 16-byte aligned, at least
+ *     fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits) bytes, not
+ *     overlapping any other argument; may be NULL when num_splits == 1. Its
+ *     contents need no initialisation and are scratch after the call returns;
+ *     two calls in flight at once must not share it.
+ * Errors as in fa_fwd; additionally Nq > Nk, num_splits out of range or a
+ * missing/short/misaligned workspace return FA_ERR_INVALID_ARG.
+ */
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int H, int H_kv, int Nq, int Nk, int d, float scale,
+                   int causal, const int32_t *kv_len, int num_splits,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of workspace fa_fwd_splitkv needs: 0 for num_splits == 1, else
+ * num_splits * B * H * Nq * (d + 1) * 4 rounded up to 256 bytes in the middle.
+ * Returns 0 for invalid arguments. Host-only, no device call.
+ */
+size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits);
+
+/*
+ * A num_splits for fa_fwd_splitkv on the current device. Work units (one per
+ * head group, row block and range) are equal-sized, so this is the fewest
+ * ranges, each at least four 128-key tiles long and at most FA_MAX_SPLITS,
+ * that make at least one full wave of units over the SMs with the last wave at
+ * least 90 % full (else the best-filled count). Returns 1 for invalid
+ * arguments. Reads only device attributes.
+ */
+int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
 
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(int status);

@@ -6,10 +6,13 @@ kernels of the library. There is no CPU fallback: if the library is missing
 or the device is not an sm_100 GPU, calls fail loudly.
 
 Names follow the C ABI: :func:`fa_fwd`, :func:`fa_fwd_kvlen`, :func:`fa_fwd_gqa`,
-:func:`fa_status_string`, :func:`fa_last_device_error`,
-:func:`fa_watchdog_selftest`. :func:`attention` is a convenience wrapper that
-allocates the outputs with torch and calls :func:`fa_fwd` / :func:`fa_fwd_kvlen`
-/ :func:`fa_fwd_gqa` on the current stream.
+:func:`fa_fwd_splitkv`, :func:`fa_splitkv_workspace_bytes`,
+:func:`fa_splitkv_default_splits`, :func:`fa_status_string`,
+:func:`fa_last_device_error`, :func:`fa_watchdog_selftest`. :func:`attention`
+is a convenience wrapper that allocates the outputs with torch and calls
+:func:`fa_fwd` / :func:`fa_fwd_kvlen` / :func:`fa_fwd_gqa` on the current
+stream; :func:`decode_attention` does the same for :func:`fa_fwd_splitkv`
+(fewer queries than keys), allocating its workspace with torch.
 """
 from __future__ import annotations
 
@@ -54,6 +57,14 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd_kvlen.restype = i
     lib.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp]
     lib.fa_fwd_gqa.restype = i
+    sz = ctypes.c_size_t
+    lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz,
+                                   vp]
+    lib.fa_fwd_splitkv.restype = i
+    lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.fa_splitkv_workspace_bytes.restype = sz
+    lib.fa_splitkv_default_splits.argtypes = [i, i, i, i, i, i]
+    lib.fa_splitkv_default_splits.restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_error.argtypes = [vp]
@@ -87,6 +98,23 @@ def fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, kv_len, stream)
     """C ABI fa_fwd_gqa: k, v have H_kv heads shared by groups of H / H_kv query heads."""
     return load_library().fa_fwd_gqa(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal,
                                      kv_len, stream)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, scale, causal, kv_len,
+                   num_splits, workspace, workspace_bytes, stream) -> int:
+    """C ABI fa_fwd_splitkv: Nq query rows against Nk >= Nq keys, keys cut into
+    num_splits ranges whose partial results are merged by log-sum-exp."""
+    return load_library().fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, scale,
+                                         causal, kv_len, num_splits, workspace,
+                                         workspace_bytes, stream)
+
+
+def fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits) -> int:
+    return int(load_library().fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits))
+
+
+def fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d) -> int:
+    return int(load_library().fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d))
 
 
 def fa_status_string(status: int) -> str:
@@ -152,4 +180,49 @@ def attention(q, k, v, scale=None, causal=False, kv_len=None, out=None, lse=None
                           float(scale), int(bool(causal)), _ptr(kv_len), s)
     if check and st != FA_OK:
         raise FAError(st, "fa_fwd")
+    return out, lse
+
+
+def decode_attention(q, k, v, scale=None, causal=False, kv_len=None, num_splits=None,
+                     out=None, lse=None, workspace=None, stream=None, check=True):
+    """O, lse for bf16 CUDA tensors q [B, H, Nq, d] and k, v [B, H_kv, Nk, d]
+    with Nq <= Nk (query row i at key position i + Nk - Nq), through
+    fa_fwd_splitkv. num_splits=None takes fa_splitkv_default_splits. The
+    workspace (if any) is allocated with torch unless given as a CUDA uint8
+    tensor of at least fa_splitkv_workspace_bytes bytes.
+    """
+    import torch
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("q, k, v must be bfloat16")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors (no CPU fallback)")
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape or \
+            (q.shape[0], q.shape[3]) != (k.shape[0], k.shape[3]):
+        raise ValueError(f"q [B,H,Nq,d] and k, v [B,H_kv,Nk,d] expected, got "
+                         f"{q.shape} {k.shape} {v.shape}")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous")
+    B, H, Nq, d = q.shape
+    H_kv, Nk = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if num_splits is None:
+        num_splits = fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if kv_len is not None and (kv_len.dtype != torch.int32 or not kv_len.is_cuda
+                               or kv_len.shape != (B,)):
+        raise ValueError("kv_len must be a CUDA int32 tensor of shape [B]")
+    need = fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    s = stream if stream is not None else torch.cuda.current_stream(q.device).cuda_stream
+    st = fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, Nq, Nk,
+                        d, float(scale), int(bool(causal)), _ptr(kv_len), int(num_splits),
+                        _ptr(workspace), ws_bytes, s)
+    if check and st != FA_OK:
+        raise FAError(st, "fa_fwd_splitkv")
     return out, lse

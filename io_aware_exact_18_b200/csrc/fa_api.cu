@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_combine_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
@@ -39,6 +40,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kWatchdogNs = 1000000000ull;  // 1 s per bounded wait
 constexpr int64_t kL2GroupBytes = 80ll << 20;     // K/V bytes of one launch-order head group
+constexpr int kMaxSplits = FA_MAX_SPLITS;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -48,9 +50,16 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 struct DeviceState {
     bool probed = false;
     bool supported = false;
-    bool smem_set[3] = {false, false, false};  // d = 64, 128, 256
     uint32_t* err_ptr = nullptr;
 };
+
+// Opt in to the dynamic shared memory of one kernel instantiation.
+template <int D, int QT, bool kGen>
+bool set_smem() {
+    return cudaFuncSetAttribute(fa_fwd_sm100<D, QT, kGen>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<D, QT>::kSmemBytes) == cudaSuccess;
+}
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
@@ -69,8 +78,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // Device set-up (once per device, under the lock): capability check, the
-// address of the status word, the opt-in shared-memory size.
-int prepare_device(int d, int* dev_out, uint32_t** err_out) {
+// address of the status word, the opt-in shared-memory size of every kernel.
+int prepare_device(int* dev_out, uint32_t** err_out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
@@ -86,39 +95,30 @@ int prepare_device(int d, int* dev_out, uint32_t** err_out) {
             void* p = nullptr;
             if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return FA_ERR_LAUNCH;
             st.err_ptr = static_cast<uint32_t*>(p);
+            const bool ok = set_smem<64, 2, false>() && set_smem<128, 2, false>() &&
+                            set_smem<256, 1, false>() && set_smem<64, 1, true>() &&
+                            set_smem<128, 1, true>() && set_smem<256, 1, true>();
+            if (!ok) return FA_ERR_LAUNCH;
         }
         st.probed = true;
     }
     if (!st.supported) return FA_ERR_UNSUPPORTED;
-    const int di = (d == 256) ? 2 : (d == 128) ? 1 : 0;
-    if (!st.smem_set[di]) {
-        cudaError_t e =
-            (d == 256) ? cudaFuncSetAttribute(fa_fwd_sm100<256>,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              Cfg<256>::kSmemBytes)
-            : (d == 128) ? cudaFuncSetAttribute(fa_fwd_sm100<128>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                Cfg<128>::kSmemBytes)
-                         : cudaFuncSetAttribute(fa_fwd_sm100<64>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                Cfg<64>::kSmemBytes);
-        if (e != cudaSuccess) return FA_ERR_LAUNCH;
-        st.smem_set[di] = true;
-    }
     *dev_out = dev;
     *err_out = st.err_ptr;
     return FA_OK;
 }
 
 // 3-D view [B*H, N, d] of a contiguous bf16 tensor; box = 64 columns (128
-// bytes, the swizzle width) x 128 rows x 1 head. The third dimension keeps a
-// tile from ever crossing into the next head: rows past N read as zero.
-int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+// bytes, the swizzle width) x box_rows rows x box_planes heads. The third
+// dimension keeps a tile from ever crossing into the next head: rows past N
+// read as zero.
+int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows = 128,
+             int box_planes = 1) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return FA_ERR_LAUNCH;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_planes};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -132,77 +132,180 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
-int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int H_kv, int N, int d, float scale, int causal, const int32_t* kv_len,
-             void* stream) {
+// One forward call. Q [B,H,Nq,d]; K, V [B,H_kv,Nk,d]; O [B,H,Nq,d]; lse
+// [B,H,Nq]. splits > 1 writes per-range partials into `ws` and merges them.
+struct FwdCall {
+    const void *q, *k, *v;
+    void* o;
+    float* lse;
+    int B, H, H_kv, Nq, Nk, d;
+    float scale;
+    int causal;
+    const int32_t* kv_len;
+    int splits;          // >= 1
+    bool pack;           // pack the query heads of a K/V group into one tile
+    void* ws;            // split partials (splits > 1)
+    size_t ws_bytes;
+};
+
+// Workspace layout for `splits` ranges: O partials fp32 [splits][B*H][Nq][d],
+// then (256-byte aligned) lse partials fp32 [splits][B*H][Nq].
+size_t ws_o_bytes(int64_t rows, int d, int splits) {
+    const size_t b = (size_t)splits * (size_t)rows * (size_t)d * 4;
+    return (b + 255) & ~size_t(255);
+}
+size_t ws_total_bytes(int64_t rows, int d, int splits) {
+    if (splits <= 1) return 0;
+    return ws_o_bytes(rows, d, splits) + (size_t)splits * (size_t)rows * 4;
+}
+
+// Query heads per tile and rows per head in a tile.
+void tile_shape(int H, int H_kv, int Nq, bool pack, int* G, int* nq_blk) {
+    const int grp = H / H_kv;
+    if (pack && grp > 1 && grp <= kTile) {
+        *G = grp;
+        *nq_blk = std::min(Nq, kTile / grp);
+    } else {
+        *G = 1;
+        *nq_blk = kTile;
+    }
+}
+
+int fwd_impl(const FwdCall& a, void* stream) {
     // ---- arguments (synchronous, nothing launched on error)
-    if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+    const int B = a.B, H = a.H, H_kv = a.H_kv, Nq = a.Nq, Nk = a.Nk, d = a.d;
+    if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || Nq > Nk) return FA_ERR_INVALID_ARG;
     if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_INVALID_ARG;
-    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (a.causal != 0 && a.causal != 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(a.scale) || !(a.scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (a.splits < 1 || a.splits > kMaxSplits) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-    if (B == 0 || H == 0 || N == 0) return FA_OK;
-    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-    const uintptr_t a16 = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
-    if ((a16 & 15u) != 0 || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    if (B == 0 || H == 0 || Nq == 0) return FA_OK;
+    if (!a.q || !a.k || !a.v || !a.o || !a.lse) return FA_ERR_INVALID_ARG;
+    const uintptr_t a16 = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
+                          reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(a.o);
+    if ((a16 & 15u) != 0 || (reinterpret_cast<uintptr_t>(a.lse) & 3u) != 0)
         return FA_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0) return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(a.kv_len) & 3u) != 0) return FA_ERR_INVALID_ARG;
     const int64_t BH = (int64_t)B * H;
     const int64_t BHkv = (int64_t)B * H_kv;
-    const int64_t rows_per_unit = (d == 256) ? 128 : 256;   // query tiles per unit x 128
-    const int64_t n_units = ((int64_t)N + rows_per_unit - 1) / rows_per_unit;
-    if (BH > INT32_MAX || BH * n_units > INT32_MAX) return FA_ERR_INVALID_ARG;
-    const size_t elems = (size_t)BH * (size_t)N * (size_t)d;
-    if ((double)BH * N * d > 9.0e18) return FA_ERR_INVALID_ARG;
-    const size_t tbytes = elems * 2, lbytes = (size_t)BH * (size_t)N * 4;
-    const size_t kvbytes = (size_t)BHkv * (size_t)N * (size_t)d * 2;
-    if (overlaps(o, tbytes, q, tbytes) || overlaps(o, tbytes, k, kvbytes) ||
-        overlaps(o, tbytes, v, kvbytes) || overlaps(lse, lbytes, q, tbytes) ||
-        overlaps(lse, lbytes, k, kvbytes) || overlaps(lse, lbytes, v, kvbytes) ||
-        overlaps(lse, lbytes, o, tbytes))
+    int G = 1, nq_blk = kTile;
+    tile_shape(H, H_kv, Nq, a.pack, &G, &nq_blk);
+    // Square attention (one key range, no packing, Nq == Nk) runs the
+    // specialised kernels; everything else the general one-query-tile kernel.
+    const bool general = a.splits > 1 || G > 1 || Nq != Nk;
+    const int qt = (general || d == 256) ? 1 : 2;          // query tiles per unit
+    const int64_t n_rb = ((int64_t)Nq + nq_blk - 1) / nq_blk;
+    const int64_t n_units = (n_rb + qt - 1) / qt * a.splits;
+    const int64_t BHB = BH / G;
+    if (BH > INT32_MAX || BHB * n_units > INT32_MAX) return FA_ERR_INVALID_ARG;
+    if ((double)BH * Nq * d > 9.0e18 || (double)BHkv * Nk * d > 9.0e18) return FA_ERR_INVALID_ARG;
+    const int64_t rows = BH * Nq;
+    if (rows > INT32_MAX) return FA_ERR_INVALID_ARG;      // row indices are 32-bit in the kernel
+    const size_t tbytes = (size_t)rows * d * 2, lbytes = (size_t)rows * 4;
+    const size_t kvbytes = (size_t)BHkv * (size_t)Nk * (size_t)d * 2;
+    if (overlaps(a.o, tbytes, a.q, tbytes) || overlaps(a.o, tbytes, a.k, kvbytes) ||
+        overlaps(a.o, tbytes, a.v, kvbytes) || overlaps(a.lse, lbytes, a.q, tbytes) ||
+        overlaps(a.lse, lbytes, a.k, kvbytes) || overlaps(a.lse, lbytes, a.v, kvbytes) ||
+        overlaps(a.lse, lbytes, a.o, tbytes))
         return FA_ERR_INVALID_ARG;
+    float* o_part = nullptr;
+    float* lse_part = nullptr;
+    if (a.splits > 1) {
+        const size_t need = ws_total_bytes(rows, d, a.splits);
+        if (a.ws == nullptr || a.ws_bytes < need || (reinterpret_cast<uintptr_t>(a.ws) & 15u) != 0)
+            return FA_ERR_INVALID_ARG;
+        if (overlaps(a.ws, need, a.q, tbytes) || overlaps(a.ws, need, a.k, kvbytes) ||
+            overlaps(a.ws, need, a.v, kvbytes) || overlaps(a.ws, need, a.o, tbytes) ||
+            overlaps(a.ws, need, a.lse, lbytes))
+            return FA_ERR_INVALID_ARG;
+        o_part = static_cast<float*>(a.ws);
+        lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
+                                            ws_o_bytes(rows, d, a.splits));
+    }
 
     int dev = 0;
     uint32_t* err = nullptr;
-    int rc = prepare_device(d, &dev, &err);
+    int rc = prepare_device(&dev, &err);
     if (rc != FA_OK) return rc;
 
     alignas(64) CUtensorMap mq, mk, mv;
-    if ((rc = make_map(&mq, q, (int)BH, N, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mk, k, (int)BHkv, N, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, v, (int)BHkv, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mq, a.q, (int)BH, Nq, d, nq_blk, G)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, a.k, (int)BHkv, Nk, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, a.v, (int)BHkv, Nk, d)) != FA_OK) return rc;
 
     FwdParams p{};
-    p.o = static_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.kv_len = kv_len;
+    p.o = static_cast<__nv_bfloat16*>(a.o);
+    p.lse = a.lse;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.kv_len = a.kv_len;
     p.dev_err = err;
     p.B = B;
     p.H = H;
     p.H_kv = H_kv;
-    p.N = N;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.q_off = Nk - Nq;
+    p.G = G;
+    p.nq_blk = nq_blk;
+    p.n_rb = (int)n_rb;
+    p.splits = a.splits;
     p.n_units = (int)n_units;
-    // Launch-order head groups: as few groups as keep a group's K/V (2*N*d*2
-    // bytes per K/V head, shared by H / H_kv query heads) within
-    // kL2GroupBytes, with the query heads split evenly.
-    const int64_t kv_head_bytes = (int64_t)N * d * 4;
-    const int64_t cap = std::max<int64_t>(1, kL2GroupBytes / kv_head_bytes) * (H / H_kv);
-    const int64_t groups = (BH + cap - 1) / cap;
-    p.group_heads = (int)((BH + groups - 1) / groups);
-    p.causal = causal;
-    p.scale_log2 = scale * 1.4426950408889634f;
+    // Launch-order head groups: as few groups as keep a group's K/V (2*Nk*d*2
+    // bytes per K/V head, shared by H / H_kv query heads, G of them per head
+    // block) within kL2GroupBytes, with the head blocks split evenly.
+    const int64_t kv_head_bytes = (int64_t)Nk * d * 4;
+    const int64_t cap =
+        std::max<int64_t>(1, kL2GroupBytes / kv_head_bytes) * ((H / H_kv) / G);
+    const int64_t groups = (BHB + cap - 1) / cap;
+    p.group_heads = (int)((BHB + groups - 1) / groups);
+    p.causal = a.causal;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
     p.watchdog_ns = kWatchdogNs;
 
-    const dim3 grid((unsigned)(BH * n_units)), block(kThreads);
+    const dim3 grid((unsigned)(BHB * n_units)), block(kThreads);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 256)
-        fa_fwd_sm100<256><<<grid, block, Cfg<256>::kSmemBytes, s>>>(mq, mk, mv, p);
-    else if (d == 128)
-        fa_fwd_sm100<128><<<grid, block, Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
-    else
-        fa_fwd_sm100<64><<<grid, block, Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
-    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+    if (general) {
+        if (d == 256)
+            fa_fwd_sm100<256, 1, true><<<grid, block, Cfg<256, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else if (d == 128)
+            fa_fwd_sm100<128, 1, true><<<grid, block, Cfg<128, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else
+            fa_fwd_sm100<64, 1, true><<<grid, block, Cfg<64, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+    } else {
+        if (d == 256)
+            fa_fwd_sm100<256, 1, false><<<grid, block, Cfg<256, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else if (d == 128)
+            fa_fwd_sm100<128, 2, false><<<grid, block, Cfg<128, 2>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else
+            fa_fwd_sm100<64, 2, false><<<grid, block, Cfg<64, 2>::kSmemBytes, s>>>(mq, mk, mv, p);
+    }
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+    if (a.splits > 1) {
+        const dim3 cgrid((unsigned)((rows + kCombineWarps - 1) / kCombineWarps));
+        const dim3 cblock(32 * kCombineWarps);
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
+        if (d == 256)
+            fa_splitkv_combine<256><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits);
+        else if (d == 128)
+            fa_splitkv_combine<128><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits);
+        else
+            fa_splitkv_combine<64><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
+FwdCall square_call(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int H_kv, int N, int d, float scale, int causal,
+                    const int32_t* kv_len) {
+    FwdCall a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.H = H; a.H_kv = H_kv; a.Nq = N; a.Nk = N; a.d = d;
+    a.scale = scale; a.causal = causal; a.kv_len = kv_len;
+    a.splits = 1; a.pack = false; a.ws = nullptr; a.ws_bytes = 0;
+    return a;
 }
 
 }  // namespace
@@ -214,19 +317,71 @@ extern "C" {
 
 FA_EXPORT int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
            int d, float scale, int causal, void* stream) {
-    return fa::fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, nullptr, stream);
+    return fa::fwd_impl(fa::square_call(q, k, v, o, lse, B, H, H, N, d, scale, causal, nullptr),
+                        stream);
 }
 
 FA_EXPORT int fa_fwd_kvlen(const void* q, const void* k, const void* v, void* o, float* lse,
                            int B, int H, int N, int d, float scale, int causal,
                            const int32_t* kv_len, void* stream) {
-    return fa::fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, kv_len, stream);
+    return fa::fwd_impl(fa::square_call(q, k, v, o, lse, B, H, H, N, d, scale, causal, kv_len),
+                        stream);
 }
 
 FA_EXPORT int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
                          int B, int H, int H_kv, int N, int d, float scale, int causal,
                          const int32_t* kv_len, void* stream) {
-    return fa::fwd_impl(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, kv_len, stream);
+    return fa::fwd_impl(
+        fa::square_call(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, kv_len), stream);
+}
+
+FA_EXPORT size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits) {
+    if (B < 0 || H < 0 || Nq < 0 || d < 0 || num_splits < 1 || num_splits > fa::kMaxSplits)
+        return 0;
+    return fa::ws_total_bytes((int64_t)B * H * Nq, d, num_splits);
+}
+
+FA_EXPORT int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d) {
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Nq < 1 || Nk < 1) return 1;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    int G = 1, nq_blk = fa::kTile;
+    fa::tile_shape(H, H_kv, Nq, true, &G, &nq_blk);
+    (void)d;   // one query tile per unit at every d
+    const int64_t n_rb = ((int64_t)Nq + nq_blk - 1) / nq_blk;
+    const int64_t base = (int64_t)B * (H / G) * n_rb;
+    const int64_t key_tiles = ((int64_t)Nk + fa::kTile - 1) / fa::kTile;
+    // Units are equal-sized, so the last wave decides: take the fewest ranges
+    // (each at least four key tiles) that give at least one full wave of
+    // units with the last wave >= 90 % busy; else the best-filled count.
+    const int64_t s_max = std::min<int64_t>(fa::kMaxSplits, std::max<int64_t>(1, key_tiles / 4));
+    int64_t best = 1;
+    double best_eff = -1.0;
+    for (int64_t sp = 1; sp <= s_max; ++sp) {
+        const int64_t units = base * sp;
+        const int64_t waves = (units + sms - 1) / sms;
+        const double eff = (double)units / (double)(waves * sms);
+        if (units >= sms && eff >= 0.9) return (int)sp;
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = sp;
+        }
+    }
+    return (int)best;
+}
+
+FA_EXPORT int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int H_kv, int Nq, int Nk, int d, float scale,
+                             int causal, const int32_t* kv_len, int num_splits, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    fa::FwdCall a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.H = H; a.H_kv = H_kv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+    a.scale = scale; a.causal = causal; a.kv_len = kv_len;
+    a.splits = num_splits; a.pack = true; a.ws = workspace; a.ws_bytes = workspace_bytes;
+    return fa::fwd_impl(a, stream);
 }
 
 FA_EXPORT const char* fa_status_string(int status) {
@@ -244,7 +399,7 @@ FA_EXPORT int fa_watchdog_selftest(uint64_t limit_ns, void* stream) {
     if (limit_ns < 1000ull || limit_ns > 5000000000ull) return FA_ERR_INVALID_ARG;
     int dev = 0;
     uint32_t* err = nullptr;
-    const int rc = fa::prepare_device(64, &dev, &err);
+    const int rc = fa::prepare_device(&dev, &err);
     if (rc != FA_OK) return rc;
     fa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_ns);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;

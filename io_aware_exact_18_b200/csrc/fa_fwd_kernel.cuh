@@ -21,8 +21,14 @@
 // stays below 2^64, far inside the fp32 and bf16 range.
 //
 // Work partitioning ("FlashAttention-2 (HI)", sections 2 and 3). A work unit
-// is one (batch, head, pair of 128-row query tiles); the grid has one CTA per
-// unit, so one long head still spreads over every SM. Units are numbered in
+// is one (batch, head, pair of 128-row query tiles) -- one tile at d = 256 --
+// and the grid has one CTA per unit, so one long head still spreads over every
+// SM. The general instantiation (kGen) adds what decoding against a key-value
+// cache needs ("FlashAttention (UR)", section "Specialised solutions"): fewer
+// query rows than keys (row i at key position i + Nk - Nq), the query heads of
+// a K/V group packed into one tile so each K/V tile serves all of them, and
+// units that take one range of key tiles each, writing a normalised partial O
+// and lse for a separate merge (split-KV). Units are numbered in
 // launch order: heads in groups whose K/V fit in L2 together, and within a
 // group the query-tile pairs heaviest first (the last pairs, for causal
 // masking) across the group's heads. CTAs are persistent: near the end of
@@ -80,19 +86,24 @@ constexpr int kTmaWarp = 9;
 constexpr float kMaxTileSum = 18446744073709551616.0f;  // 2^64
 constexpr float kLn2 = 0.69314718055994530942f;
 
-// Per head dimension. d = 64, 128: a unit is two query tiles, each with one
-// S buffer (TMEM: S0 | S1 | O0 | O1). d = 256: O alone takes 256 TMEM columns,
-// so a unit is one query tile whose S is double-buffered (TMEM: Sa | Sb | O):
-// the tensor cores compute the next tile's scores while the softmax works on
-// the current ones, and at d = 256 each key tile carries twice the MMA work.
-template <int D>
+// Per head dimension and query tiles per unit. QT = 2 (square attention at
+// d = 64, 128): a unit is two query tiles, each with one S buffer (TMEM:
+// S0 | S1 | O0 | O1), and the two softmax warpgroups ping-pong. QT = 1: a unit
+// is one query tile whose S is double-buffered (TMEM: Sa | Sb | O): the tensor
+// cores compute the next key tile's scores while the softmax works on the
+// current ones. d = 256 needs it (O alone takes 256 TMEM columns); the
+// split-KV kernel uses it at every d, since a short query block gives the
+// second tile of a pair nothing to do.
+template <int D, int QT>
 struct Cfg {
     static_assert(D == 64 || D == 128 || D == 256, "head dim 64, 128 or 256");
-    static constexpr int kQT = (D == 256) ? 1 : 2;        // query tiles per unit
+    static_assert(QT == 1 || (QT == 2 && D <= 128), "two query tiles need d <= 128");
+    static constexpr int kQT = QT;                        // query tiles per unit
     static constexpr int kBlocks = D / 64;                // 128-byte column blocks per row
     static constexpr int kBlockBytes = kTile * 128;       // 16 KB
     static constexpr int kTileBytes = kTile * D * 2;      // one Q/K/V tile
-    static constexpr int kSlots = (D == 256) ? 2 : (D == 128) ? 4 : 8;  // K/V ring depth
+    static constexpr int kSlots =                         // K/V ring depth
+        (D == 256) ? 2 : (D == 128) ? (QT == 2 ? 4 : 5) : 8;
     static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 1024 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
@@ -106,14 +117,22 @@ struct Cfg {
 };
 
 struct FwdParams {
-    __nv_bfloat16* o;          // [B,H,N,d]
-    float* lse;                // [B,H,N]
+    __nv_bfloat16* o;          // [B,H,Nq,d]
+    float* lse;                // [B,H,Nq]
+    float* o_part;             // split-KV partials [splits][B*H][Nq][d] fp32, or nullptr
+    float* lse_part;           // [splits][B*H][Nq]
     const int32_t* kv_len;     // [B] or nullptr
     uint32_t* dev_err;         // status word
-    int B, H, N;
+    int B, H;
     int H_kv;                  // K/V heads; query head h reads K/V head h / (H / H_kv)
-    int n_units;               // units per head: ceil(N / (128 * query tiles per unit))
-    int group_heads;           // heads per L2 group (launch order)
+    int Nq, Nk;                // query rows, keys
+    int q_off;                 // causal offset: query row i stands at key position i + q_off
+    int G;                     // query heads packed into one tile (they share a K/V head)
+    int nq_blk;                // query rows per head in one tile (G * nq_blk <= 128)
+    int n_rb;                  // row blocks per head: ceil(Nq / nq_blk)
+    int splits;                // key ranges per row block (1 = no split)
+    int n_units;               // units per head block: ceil(n_rb / query tiles per unit) * splits
+    int group_heads;           // head blocks per L2 group (launch order)
     int causal;
     float scale_log2;          // scale * log2(e)
     uint64_t watchdog_ns;
@@ -141,39 +160,71 @@ struct SmemBarriers {
 static_assert(sizeof(SmemBarriers) <= 1024, "barrier region");
 static_assert(offsetof(SmemBarriers, clc_resp) % 16 == 0, "CLC response alignment");
 
-// One work unit, decoded from its launch-order index.
+// One work unit, decoded from its launch-order index. A tile's 128 rows hold
+// G heads x nq_blk query rows (row r: head h0 + r / nq_blk, query row
+// q_first + r % nq_blk); with G = 1, nq_blk = 128 a tile is 128 rows of one head.
 struct Unit {
-    int bh, b, q0, kv_lim;
-    int bkv;                   // K/V head row in the [B*H_kv, N, d] view
+    int b, h0;                 // batch, first query head of the tile
+    int bkv;                   // K/V head row in the [B*H_kv, Nk, d] view
+    int rb0;                   // row block of query tile 0 (tile t: rb0 + t)
+    int s, kt0;                // split index and its first key tile
+    int kv_lim;
     int n[2];                  // key tiles each query tile visits (0 = idle tile)
     int n_max;
 };
 
-// Number of 128-key tiles a query tile starting at row q_first must visit.
-__device__ __forceinline__ int kv_tiles_for(int q_first, int N, int kv_lim, int causal) {
-    if (q_first >= N) return 0;
+// Tile-shape parameters: read from FwdParams by the general (split-KV,
+// packed-heads, Nq <= Nk) kernel, compile-time constants for square attention
+// (one head of 128 rows per tile, one key range, Nq == Nk).
+template <bool kGen>
+struct Shape {
+    int G, nq_blk, splits, q_off, Nq;
+    __device__ __forceinline__ explicit Shape(const FwdParams& p)
+        : G(kGen ? p.G : 1),
+          nq_blk(kGen ? p.nq_blk : kTile),
+          splits(kGen ? p.splits : 1),
+          q_off(kGen ? p.q_off : 0),
+          Nq(kGen ? p.Nq : p.Nk) {}
+};
+
+// Key tiles a row block must visit: keys below its last row's causal limit
+// (key position of the row + 1) and below kv_lim.
+template <bool kGen>
+__device__ __forceinline__ int kv_tiles_for(int rb, const FwdParams& p, const Shape<kGen>& sh,
+                                            int kv_lim) {
+    const int q_first = rb * sh.nq_blk;
+    if (q_first >= sh.Nq) return 0;
     int lim = kv_lim;
-    if (causal) lim = min(lim, q_first + kTile);
-    return (lim + kTile - 1) / kTile;
+    if (p.causal) lim = min(lim, min(q_first + sh.nq_blk, sh.Nq) + sh.q_off);
+    return (max(lim, 0) + kTile - 1) / kTile;
 }
 
-template <int QT>
+template <int QT, bool kGen>
 __device__ __forceinline__ Unit decode_unit(int id, const FwdParams& p) {
+    const Shape<kGen> sh(p);
     Unit u;
-    const int BH = p.B * p.H;
+    const int hpb = p.H / sh.G;                // head blocks per batch
+    const int BHB = p.B * hpb;
     const int per_group = p.group_heads * p.n_units;
     const int grp = id / per_group;
     const int in_grp = id - grp * per_group;
-    const int heads_here = min(p.group_heads, BH - grp * p.group_heads);
-    const int pair = p.n_units - 1 - in_grp / heads_here;
-    u.bh = grp * p.group_heads + in_grp % heads_here;
-    u.b = u.bh / p.H;
-    u.bkv = u.b * p.H_kv + (u.bh - u.b * p.H) / (p.H / p.H_kv);
-    u.q0 = pair * QT * kTile;
-    u.kv_lim = p.N;
-    if (p.kv_len != nullptr) u.kv_lim = max(0, min(p.N, p.kv_len[u.b]));
-    u.n[0] = kv_tiles_for(u.q0, p.N, u.kv_lim, p.causal);
-    u.n[1] = (QT == 2) ? kv_tiles_for(u.q0 + kTile, p.N, u.kv_lim, p.causal) : 0;
+    const int heads_here = min(p.group_heads, BHB - grp * p.group_heads);
+    const int ps = p.n_units - 1 - in_grp / heads_here;   // (row-block pair, split), heaviest first
+    const int hb = grp * p.group_heads + in_grp % heads_here;
+    u.b = hb / hpb;
+    u.h0 = (hb - u.b * hpb) * sh.G;
+    u.bkv = u.b * p.H_kv + u.h0 / (p.H / p.H_kv);
+    const int pair = ps / sh.splits;
+    u.s = ps - pair * sh.splits;
+    u.rb0 = pair * QT;
+    u.kv_lim = p.Nk;
+    if (p.kv_len != nullptr) u.kv_lim = max(0, min(p.Nk, p.kv_len[u.b]));
+    // split s takes key tiles [s * nkb / splits, (s + 1) * nkb / splits)
+    const int nkb = (u.kv_lim + kTile - 1) / kTile;
+    u.kt0 = kGen ? (int)((long long)u.s * nkb / sh.splits) : 0;
+    const int kt1 = kGen ? (int)((long long)(u.s + 1) * nkb / sh.splits) : nkb;
+    u.n[0] = max(0, min(kv_tiles_for(u.rb0, p, sh, u.kv_lim), kt1) - u.kt0);
+    u.n[1] = (QT == 2) ? max(0, min(kv_tiles_for(u.rb0 + 1, p, sh, u.kv_lim), kt1) - u.kt0) : 0;
     u.n_max = max(u.n[0], u.n[1]);
     return u;
 }
@@ -212,11 +263,12 @@ __device__ __forceinline__ float exp_tile(const float (&s)[kTile], float c, floa
     return sum0 + sum1;
 }
 
-template <int D>
+template <int D, int QT, bool kGen>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = Cfg<D>;
+    using C = Cfg<D, QT>;
+    const Shape<kGen> sh(p);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -272,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint64_t pol_kv = policy_evict_last();
             const uint64_t pol_q = policy_evict_first();
+            const uint32_t q_bytes = (uint32_t)(C::kBlocks * sh.G * sh.nq_blk * 128);
             int id = skip ? -1 : (int)blockIdx.x;
             int L = 0;                 // K/V loads issued (K_j and V_j of every unit, in order)
             int k = 0;                 // units published
@@ -312,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
                 for (int blk = 0; blk < C::kBlocks; ++blk)
                     tma_load_3d_hint(map, &bars->kv_full[slot], dst + blk * C::kBlockBytes,
-                                     blk * 64, tile * kTile, u.bkv, pol_kv);
+                                     blk * 64, (u.kt0 + tile) * kTile, u.bkv, pol_kv);
                 ++L;
                 return true;
             };
@@ -323,21 +376,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bars->unit_id[us] = id;
                 mbar_arrive(&bars->unit_full[us]);
                 if (id < 0) break;
-                const Unit u = decode_unit<C::kQT>(id, p);
+                const Unit u = decode_unit<C::kQT, kGen>(id, p);
                 // The first two K/V loads go first: the ring has room while the
                 // previous unit's last tiles are consumed, and Q may have to wait.
                 const int early = min(2, 2 * u.n_max);
                 for (int jj = 0; ok && jj < early; ++jj) ok = load_kv(u, jj);
-                // Q tiles (one q_full phase per unit and tile, possibly with no bytes)
+                // Q tiles (one q_full phase per unit and tile, possibly with no
+                // bytes). One box per 64-column block: nq_blk rows of G heads.
                 for (int t = 0; t < C::kQT && ok; ++t) {
                     if (k > 0) ok = mbar_wait(&bars->q_empty[t], (uint32_t)((k - 1) & 1), wd);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&bars->q_full[t], u.n[t] > 0 ? C::kTileBytes : 0);
+                    mbar_arrive_expect_tx(&bars->q_full[t], u.n[t] > 0 ? q_bytes : 0u);
                     q_unit[t] = k;
                     if (u.n[t] > 0)
                         for (int blk = 0; blk < C::kBlocks; ++blk)
                             tma_load_3d_hint(&tm_q, &bars->q_full[t], sQ[t] + blk * C::kBlockBytes,
-                                             blk * 64, u.q0 + t * kTile, u.bh, pol_q);
+                                             blk * 64, (u.rb0 + t) * sh.nq_blk,
+                                             u.b * p.H + u.h0, pol_q);
                 }
                 // the rest of K_0, V_0, K_1, V_1, ... of this unit
                 for (int jj = early; ok && jj < 2 * u.n_max; ++jj) ok = load_kv(u, jj);
@@ -416,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int id = bars->unit_id[us];
                 mbar_arrive(&bars->unit_empty[us]);
                 if (id < 0) break;
-                const Unit u = decode_unit<C::kQT>(id, p);
+                const Unit u = decode_unit<C::kQT, kGen>(id, p);
                 // O_t is free once the previous unit's epilogue has read it
                 bool o_ready[2] = {k == 0, k == 0};
                 for (int t = 0; t < 2 && ok; ++t)
@@ -492,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int id = bars->unit_id[us];
                 mbar_arrive(&bars->unit_empty[us]);
                 if (id < 0) break;
-                const Unit u = decode_unit<C::kQT>(id, p);
+                const Unit u = decode_unit<C::kQT, kGen>(id, p);
                 const int n = u.n[0];
                 bool o_ready = (k == 0);
                 // positions of K_t and V_j in this unit's load order (see the producer)
@@ -572,10 +627,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->unit_empty[us]);
             if (id < 0) break;
-            const Unit u = decode_unit<C::kQT>(id, p);
+            const Unit u = decode_unit<C::kQT, kGen>(id, p);
             const int n = u.n[t];
-            const int i = u.q0 + t * kTile + row;     // global query row
-            const int lim_row = p.causal ? min(u.kv_lim, i + 1) : u.kv_lim;  // visible: j < lim_row
+            int row_id;    // (b*H + h)*Nq + i of this thread's row, -1 for a padding row
+            int lim_rel;   // visible keys j < lim_rel + kt0*128 (padding rows see none)
+            {
+                const int g = row / sh.nq_blk;        // head within the tile
+                const int i = (u.rb0 + t) * sh.nq_blk + (row - g * sh.nq_blk);   // query row
+                const bool valid = g < sh.G && i < sh.Nq;
+                row_id = valid ? (u.b * p.H + u.h0 + g) * sh.Nq + i : -1;
+                const int lim_row =
+                    !valid ? 0 : p.causal ? min(u.kv_lim, i + sh.q_off + 1) : u.kv_lim;
+                lim_rel = lim_row - u.kt0 * kTile;
+            }
+            // A warp whose 32 rows are all padding (packed or short query
+            // blocks) keeps every barrier hand-off but skips the arithmetic;
+            // its rows of P and O are never read back.
+            const bool idle_warp = kGen && !__any_sync(0xffffffffu, row_id >= 0);
             float m_ref = -INFINITY;   // reference maximum (raw score units)
             float l = 0.f;             // running sum of exp2((s - m_ref) * c)
 
@@ -586,6 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++ph_s[sb];
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
+                if (idle_warp) {
+                    mbar_arrive(&bars->p_full[sb]);
+                    continue;
+                }
                 tc_fence_after();
                 float s[kTile];
 #pragma unroll
@@ -597,8 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_wait_ld();
                 const int j0 = j * kTile;
-                if (j0 + kTile > lim_row) {
-                    const int lim = lim_row - j0;
+                if (j0 + kTile > lim_rel) {
+                    const int lim = lim_rel - j0;
 #pragma unroll
                     for (int q = 0; q < kTile; ++q)
                         if (q >= lim) s[q] = -INFINITY;
@@ -668,13 +740,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const bool write = i < p.N;
+            const bool write = row_id >= 0;
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = p.o + ((size_t)u.bh * p.N + (size_t)i) * D;
+            const float row_lse = (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+            const size_t orow_idx = (size_t)row_id;
+            const size_t prow_idx = (size_t)u.s * ((size_t)p.B * p.H * sh.Nq) + (size_t)row_id;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t r[32];
-                if (n > 0) {
+                if (n > 0 && !idle_warp) {
                     tmem_ld32(tO + (uint32_t)(ch * 32), r);
                     tmem_wait_ld();
                 } else {
@@ -686,8 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_before();
                     mbar_arrive(&bars->o_empty[t]);
                 }
-                if (write) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+                if (write && (!kGen || p.o_part == nullptr)) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow_idx * D + ch * 32);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint4 w;
@@ -701,11 +775,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           __uint_as_float(r[8 * v + 7]) * inv_l);
                         dst[v] = w;
                     }
+                } else if (write) {
+                    // split-KV partial: this key range's O / l in fp32
+                    float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * D + ch * 32);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        dst[v] = make_float4(__uint_as_float(r[4 * v + 0]) * inv_l,
+                                             __uint_as_float(r[4 * v + 1]) * inv_l,
+                                             __uint_as_float(r[4 * v + 2]) * inv_l,
+                                             __uint_as_float(r[4 * v + 3]) * inv_l);
                 }
             }
-            if (write)
-                p.lse[(size_t)u.bh * p.N + (size_t)i] =
-                    (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+            if (write) {
+                if (!kGen || p.o_part == nullptr) p.lse[orow_idx] = row_lse;
+                else p.lse_part[prow_idx] = row_lse;
+            }
         }
     }
 

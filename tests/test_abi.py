@@ -18,7 +18,9 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert fa.declared_symbols() == ["fa_fwd", "fa_fwd_gqa", "fa_fwd_kvlen",
-                                     "fa_last_device_error", "fa_status_string",
+                                     "fa_fwd_splitkv", "fa_last_device_error",
+                                     "fa_splitkv_default_splits",
+                                     "fa_splitkv_workspace_bytes", "fa_status_string",
                                      "fa_watchdog_selftest"]
 
 
@@ -116,3 +118,57 @@ def test_python_wrapper_refuses_cpu_tensors():
     with pytest.raises(TypeError):
         fa.attention(x.float(), x.float(), x.float())
     assert math.isclose(1 / math.sqrt(64), 0.125)
+
+
+# ---------------------------------------------------------------- split-KV
+WS = P + (6 << 30)
+SK = dict(q=P, k=P + (1 << 30), v=P + (2 << 30), o=P + (3 << 30), lse=P + (4 << 30),
+          B=2, H=8, H_kv=2, Nq=3, Nk=1000, d=128, scale=0.088, causal=1, kv_len=None,
+          splits=4, ws=WS, ws_bytes=1 << 30)
+
+
+def call_splitkv(lib, **over):
+    a = dict(SK, **over)
+    return lib.fa_fwd_splitkv(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"],
+                              a["H_kv"], a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"],
+                              a["kv_len"], a["splits"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(Nq=1001), fa.FA_ERR_INVALID_ARG),          # more queries than keys
+    (dict(Nq=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(Nk=-1, Nq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=0), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=129), fa.FA_ERR_INVALID_ARG),        # above FA_MAX_SPLITS
+    (dict(ws=0), fa.FA_ERR_INVALID_ARG),              # splits > 1 needs a workspace
+    (dict(ws_bytes=1000), fa.FA_ERR_INVALID_ARG),     # too small
+    (dict(ws=WS + 8), fa.FA_ERR_INVALID_ARG),         # misaligned
+    (dict(ws=P + (3 << 30)), fa.FA_ERR_INVALID_ARG),  # overlaps o
+    (dict(H_kv=3), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(causal=2), fa.FA_ERR_INVALID_ARG),
+    (dict(Nq=0), fa.FA_OK),                            # empty: nothing launched
+    (dict(B=0, q=0, k=0, v=0, o=0, lse=0, ws=0), fa.FA_OK),
+])
+def test_splitkv_argument_errors_are_synchronous(lib, over, status):
+    assert call_splitkv(lib, **over) == status
+
+
+def test_splitkv_workspace_bytes(lib):
+    B, H, Nq, d = 2, 8, 3, 128
+    assert lib.fa_splitkv_workspace_bytes(B, H, Nq, d, 1) == 0
+    for s in (2, 7, 128):
+        o_bytes = s * B * H * Nq * d * 4
+        o_bytes = (o_bytes + 255) // 256 * 256
+        assert lib.fa_splitkv_workspace_bytes(B, H, Nq, d, s) == o_bytes + s * B * H * Nq * 4
+    assert lib.fa_splitkv_workspace_bytes(B, H, Nq, d, 0) == 0
+    assert lib.fa_splitkv_workspace_bytes(B, H, Nq, d, 129) == 0
+    assert lib.fa_splitkv_workspace_bytes(-1, H, Nq, d, 2) == 0
+
+
+def test_splitkv_default_splits_in_range(lib):
+    for args in [(1, 32, 8, 1, 8192, 128), (64, 32, 32, 1, 512, 128), (1, 1, 1, 1, 1, 64),
+                 (1, 32, 8, 1, 1 << 20, 128)]:
+        s = lib.fa_splitkv_default_splits(*args)
+        assert 1 <= s <= 128, (args, s)
+    assert lib.fa_splitkv_default_splits(0, 32, 8, 1, 8192, 128) == 1

@@ -121,6 +121,65 @@ def make_custom(B, H, N, d, seed, q_mult=1.0, kv_len_range=None):
     return make_inputs(w, seed=seed)
 
 
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """Few query rows against a long key/value cache (split-KV path): q
+    [B, H, Nq, d], k, v [B, H_kv, Nk, d], query row i at key position
+    i + Nk - Nq."""
+    name: str
+    B: int
+    H: int
+    H_kv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool = True
+    seed: int = 11
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """4*B*H*Nq*Nk*d (every query row sees every key when Nq == 1)."""
+        return 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
+
+    def algorithmic_bytes(self) -> int:
+        """K and V read once, Q read once, O and lse written once."""
+        kv = 2 * self.B * self.H_kv * self.Nk * self.d * 2
+        qo = 2 * self.B * self.H * self.Nq * self.d * 2
+        return kv + qo + self.B * self.H * self.Nq * 4
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "B": self.B, "H": self.H, "H_kv": self.H_kv,
+                "Nq": self.Nq, "Nk": self.Nk, "d": self.d, "causal": self.causal,
+                "scale": self.scale}
+
+
+# Decoding one token per sequence against an 8K-token cache with grouped
+# K/V heads (4 query heads per K/V head), the inference setting the pages'
+# specialised kernels target ("FlashAttention (UR)", "Specialised solutions").
+DECODE_WORKLOADS = [
+    DecodeWorkload("decode_gqa_B16_H32_Hkv8_Nq1_Nk8192_d128", 16, 32, 8, 1, 8192, 128),
+]
+DECODE_BY_NAME = {w.name: w for w in DECODE_WORKLOADS}
+
+
+def make_qkv(B, H, H_kv, Nq, Nk, d, seed, kv_len_range=None):
+    """Same recipe with separate query and key counts: q [B,H,Nq,d], then k
+    and v [B,H_kv,Nk,d], then kv_len (if a range is given)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn((B, H_kv, Nk, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn((B, H_kv, Nk, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    kv_len = None
+    if kv_len_range is not None:
+        lo, hi = kv_len_range
+        kv_len = torch.randint(lo, hi + 1, (B,), generator=g).to(torch.int32)
+    return q, k, v, kv_len
+
+
 def sample_rows(N: int, seed: int, n_random: int = 256, edge: int = 128):
     """Row indices for sampled checks at full size: the first and last `edge`
     rows plus `n_random` seeded random rows, sorted and unique."""
