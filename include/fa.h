@@ -142,6 +142,35 @@ size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits);
  */
 int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
 
+/* Bytes of split-KV scratch the library itself holds on each device. */
+#define FA_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * fa_fwd_splitkv without a workspace argument, for callers that cannot
+ * allocate device memory at call time: for instance a serving loop that hands
+ * all free device memory to a key/value cache pool up front, or a C caller
+ * with no device allocator of its own. The partial results go to a scratch
+ * array of FA_STATIC_SCRATCH_BYTES (16 MiB) that the library's CUDA module
+ * reserves on each device when it is loaded; the call itself allocates
+ * nothing. The pages have no counterpart: this is an interface variant of the
+ * split-KV forward above, with the same arguments, results and errors apart
+ * from the workspace.
+ *   - The first call on a device (with that device current) looks up the
+ *     scratch's address and prepares the kernels; make it once before any
+ *     stream capture or latency-critical section.
+ *   - If fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits) exceeds
+ *     FA_STATIC_SCRATCH_BYTES the call returns FA_ERR_INVALID_ARG before any
+ *     CUDA call; use fewer splits or fa_fwd_splitkv with your own workspace.
+ *   - One scratch per device: calls that overlap on the GPU (on different
+ *     streams, or from several host threads without ordering) race on it and
+ *     give wrong results. Calls on one stream are ordered and safe.
+ *   - Nothing in the scratch has to start at zero: every partial is written
+ *     before the merge reads it.
+ */
+int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int H, int H_kv, int Nq, int Nk, int d, float scale,
+                          int causal, const int32_t *kv_len, int num_splits, void *stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char *fa_status_string(int status);
 

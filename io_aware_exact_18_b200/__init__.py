@@ -61,6 +61,9 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz,
                                    vp]
     lib.fa_fwd_splitkv.restype = i
+    lib.fa_fwd_splitkv_static.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i,
+                                          vp]
+    lib.fa_fwd_splitkv_static.restype = i
     lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.fa_splitkv_workspace_bytes.restype = sz
     lib.fa_splitkv_default_splits.argtypes = [i, i, i, i, i, i]
@@ -107,6 +110,19 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, scale, causal, kv_len
     return load_library().fa_fwd_splitkv(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, scale,
                                          causal, kv_len, num_splits, workspace,
                                          workspace_bytes, stream)
+
+
+def fa_fwd_splitkv_static(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, scale, causal, kv_len,
+                          num_splits, stream) -> int:
+    """C ABI fa_fwd_splitkv_static: fa_fwd_splitkv with the library's own
+    per-device scratch (FA_STATIC_SCRATCH_BYTES), for callers that cannot
+    allocate device memory at call time. Calls overlapping on the GPU race on
+    the one scratch."""
+    return load_library().fa_fwd_splitkv_static(q, k, v, o, lse, B, H, H_kv, Nq, Nk, d, scale,
+                                                causal, kv_len, num_splits, stream)
+
+
+FA_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 def fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits) -> int:

@@ -297,6 +297,31 @@ int fwd_impl(const FwdCall& a, void* stream) {
     return FA_OK;
 }
 
+// ------------------------------------------------------------------ static scratch
+// Split-KV scratch owned by the library, for fa_fwd_splitkv_static: callers
+// that cannot allocate device memory at call time get the partials' space from
+// this array, which the CUDA module reserves on each device when it loads.
+static __device__ __align__(256) unsigned char g_splitkv_scratch[FA_STATIC_SCRATCH_BYTES];
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Address of the current device's scratch, looked up once per device (with
+// that device current) and cached.
+int static_scratch(void** out) {
+    int dev = 0;
+    uint32_t* err = nullptr;
+    int rc = prepare_device(&dev, &err);   // capability check first
+    if (rc != FA_OK) return rc;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_splitkv_scratch) != cudaSuccess || p == nullptr)
+            return FA_ERR_LAUNCH;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return FA_OK;
+}
+
 FwdCall square_call(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int H, int H_kv, int N, int d, float scale, int causal,
                     const int32_t* kv_len) {
@@ -381,6 +406,31 @@ FA_EXPORT int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* 
     a.B = B; a.H = H; a.H_kv = H_kv; a.Nq = Nq; a.Nk = Nk; a.d = d;
     a.scale = scale; a.causal = causal; a.kv_len = kv_len;
     a.splits = num_splits; a.pack = true; a.ws = workspace; a.ws_bytes = workspace_bytes;
+    return fa::fwd_impl(a, stream);
+}
+
+FA_EXPORT int fa_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int B, int H, int H_kv, int Nq, int Nk, int d,
+                                    float scale, int causal, const int32_t* kv_len,
+                                    int num_splits, void* stream) {
+    fa::FwdCall a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.H = H; a.H_kv = H_kv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+    a.scale = scale; a.causal = causal; a.kv_len = kv_len;
+    a.splits = num_splits; a.pack = true; a.ws = nullptr; a.ws_bytes = 0;
+    // Size check first, on the host: more partials than the scratch holds is
+    // an argument error, whatever else is wrong.
+    if (B > 0 && H > 0 && Nq > 0 && num_splits >= 1 && num_splits <= fa::kMaxSplits &&
+        fa::ws_total_bytes((int64_t)B * H * Nq, d, num_splits) > (size_t)FA_STATIC_SCRATCH_BYTES)
+        return FA_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || Nq <= 0 || num_splits < 2 || num_splits > fa::kMaxSplits ||
+        (d != 64 && d != 128 && d != 256))
+        return fa::fwd_impl(a, stream);   // empty problem, argument error or no partials
+    void* scratch = nullptr;
+    const int rc = fa::static_scratch(&scratch);
+    if (rc != FA_OK) return rc;
+    a.ws = scratch;
+    a.ws_bytes = (size_t)FA_STATIC_SCRATCH_BYTES;
     return fa::fwd_impl(a, stream);
 }
 

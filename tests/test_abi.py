@@ -18,7 +18,8 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert fa.declared_symbols() == ["fa_fwd", "fa_fwd_gqa", "fa_fwd_kvlen",
-                                     "fa_fwd_splitkv", "fa_last_device_error",
+                                     "fa_fwd_splitkv", "fa_fwd_splitkv_static",
+                                     "fa_last_device_error",
                                      "fa_splitkv_default_splits",
                                      "fa_splitkv_workspace_bytes", "fa_status_string",
                                      "fa_watchdog_selftest"]
