@@ -8,6 +8,9 @@ Two independent routes to the same result:
 * :func:`attention` -- the plain definition in fp64 C (``attn_ref.c``): every
   score row is materialised in full and the softmax is taken in two passes.
   This follows "FlashAttention (UR)", section "Problem of standard attention".
+* :func:`attention_bwd` -- the gradients dQ, dK, dV of the same definition for
+  a given dO (chain rule through the row softmax, one query row at a time), in
+  fp64 C. The pages state no backward algorithm; this is the exact gradient.
 * :func:`online.attention_online` -- a blockwise online-softmax evaluation in
   numpy (running row max and running sum of exponentials, rescaled per key
   block), following section "Online softmax" of the same page. It exists only
@@ -60,6 +63,9 @@ def _bind(lib):
                                          c_int, c_int, c_int, c_int, c_double, c_int, i32p,
                                          i32p, c_int, c_int]
     lib.oracle_attn_general.restype = c_int
+    lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, u16p, u16p, u16p, u16p, dp, dp, dp, c_int,
+                                    c_int, c_int, c_int, c_int, c_double, c_int, i32p, c_int]
+    lib.oracle_attn_bwd.restype = c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     return lib
@@ -156,3 +162,46 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
     if rc != 0:
         raise RuntimeError(f"oracle returned error {rc}")
     return o, lse
+
+
+def attention_bwd(q, k, v, do, scale, causal=False, kv_len=None, nthreads=0, lib=None):
+    """Exact gradients in fp64 of attention(q, k, v) for the output gradient do.
+
+    q, do: [B, H, N, d]; k, v: [B, Hkv, N, d] (square, Nq == Nk == N; grouped
+    heads as in :func:`attention`), all bf16 torch tensors / uint16 arrays or
+    all float. Returns (dq [B,H,N,d], dk [B,Hkv,N,d], dv [B,Hkv,N,d]) float64;
+    dk and dv of a shared K/V head sum over its group of query heads.
+    """
+    lib = lib or load()
+    arrs = [_as_numpy(x) for x in (q, k, v, do)]
+    if len({b for _, b in arrs}) != 1:
+        raise TypeError("q, k, v, do must share one element type")
+    (qa, bits), (ka, _), (va, _), (da, _) = arrs
+    if qa.ndim != 4 or ka.shape != va.shape or da.shape != qa.shape:
+        raise ValueError(f"bad shapes {qa.shape} {ka.shape} {va.shape} {da.shape}")
+    B, H, N, d = qa.shape
+    Hkv = ka.shape[1]
+    if ka.shape != (B, Hkv, N, d) or Hkv < 1 or H % Hkv:
+        raise ValueError(f"bad shapes {qa.shape} {ka.shape}")
+    kvp = None
+    if kv_len is not None:
+        kvl = np.ascontiguousarray(np.asarray(
+            kv_len.cpu().numpy() if hasattr(kv_len, "cpu") else kv_len, dtype=np.int32))
+        if kvl.shape != (B,):
+            raise ValueError("kv_len must have shape [B]")
+        kvp = kvl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    dq = np.zeros((B, H, N, d), dtype=np.float64)
+    dk = np.zeros((B, Hkv, N, d), dtype=np.float64)
+    dv = np.zeros((B, Hkv, N, d), dtype=np.float64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    if bits:
+        ptrs = (None,) * 4 + tuple(a.ctypes.data_as(u16p) for a in (qa, ka, va, da))
+    else:
+        ptrs = tuple(a.ctypes.data_as(dp) for a in (qa, ka, va, da)) + (None,) * 4
+    rc = lib.oracle_attn_bwd(*ptrs, dq.ctypes.data_as(dp), dk.ctypes.data_as(dp),
+                             dv.ctypes.data_as(dp), B, H, Hkv, N, d, float(scale),
+                             int(bool(causal)), kvp, int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle returned error {rc}")
+    return dq, dk, dv

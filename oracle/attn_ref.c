@@ -262,6 +262,135 @@ int oracle_attn_general(const double *qd, const double *kd, const double *vd,
                        causal, kv_len, rows, nrows, nthreads);
 }
 
+/*
+ * Backward pass: gradients of the attention above for a scalar loss L, given
+ * dO = dL/dO. The pages report training speed-ups ("FlashAttention (UR)",
+ * section "Experimental results"), which need these gradients, but state no
+ * backward algorithm; this is the exact gradient of the forward definition by
+ * the chain rule through the row softmax, evaluated one query row at a time:
+ *   P_ij  = softmax_j(s_ij)                      (0 for hidden keys)
+ *   dV_j += P_ij dO_i                            (dV = P^T dO)
+ *   dP_ij = <dO_i, v_j>                          (dP = dO V^T)
+ *   D_i   = sum_j P_ij dP_ij
+ *   dS_ij = P_ij (dP_ij - D_i)                   (softmax Jacobian)
+ *   dQ_i  = scale sum_j dS_ij k_j                (dQ = scale dS K)
+ *   dK_j += scale dS_ij q_i                      (dK = scale dS^T Q)
+ * A K/V head shared by a group of query heads collects the sum over the
+ * group. A row with no visible key has P = 0 and contributes nothing.
+ * q, dO, dq: [B,H,N,d]; k, v, dk, dv: [B,Hkv,N,d] (square: Nq == Nk == N).
+ * Inputs fp64 (qd..dod) or bf16 bits (qb..dob), exactly one set non-null.
+ */
+static void bwd_one_row(const double *qi, const double *doi, const double *K, const double *V,
+                        int N, int d, double scale, int i, int causal, int kv_lim,
+                        double *prow, double *dsrow, double *dqi, double *dK, double *dV)
+{
+    double m = -INFINITY;
+    for (int j = 0; j < N; ++j) {
+        if (!key_allowed(i, j, causal, kv_lim, 0)) {
+            prow[j] = -INFINITY;
+            continue;
+        }
+        const double *krow = K + (size_t)j * d;
+        double dot = 0.0;
+        for (int t = 0; t < d; ++t) dot += qi[t] * krow[t];
+        prow[j] = scale * dot;
+        if (prow[j] > m) m = prow[j];
+    }
+    for (int t = 0; t < d; ++t) dqi[t] = 0.0;
+    if (m == -INFINITY) return;
+    double sum = 0.0;
+    for (int j = 0; j < N; ++j)
+        if (prow[j] != -INFINITY) sum += exp(prow[j] - m);
+    for (int j = 0; j < N; ++j)
+        prow[j] = (prow[j] == -INFINITY) ? 0.0 : exp(prow[j] - m) / sum;
+    /* dP_ij and D_i */
+    double D = 0.0;
+    for (int j = 0; j < N; ++j) {
+        if (prow[j] == 0.0) {
+            dsrow[j] = 0.0;
+            continue;
+        }
+        const double *vrow = V + (size_t)j * d;
+        double dot = 0.0;
+        for (int t = 0; t < d; ++t) dot += doi[t] * vrow[t];
+        dsrow[j] = dot;
+        D += prow[j] * dot;
+    }
+    for (int j = 0; j < N; ++j) {
+        const double pij = prow[j];
+        if (pij == 0.0) continue;
+        const double ds = pij * (dsrow[j] - D);
+        const double *krow = K + (size_t)j * d;
+        double *dkj = dK + (size_t)j * d;
+        double *dvj = dV + (size_t)j * d;
+        for (int t = 0; t < d; ++t) {
+            dqi[t] += scale * ds * krow[t];
+            dkj[t] += scale * ds * qi[t];
+            dvj[t] += pij * doi[t];
+        }
+    }
+}
+
+int oracle_attn_bwd(const double *qd, const double *kd, const double *vd, const double *dod,
+                    const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
+                    const uint16_t *dob, double *dq, double *dk, double *dv, int B, int H,
+                    int Hkv, int N, int d, double scale, int causal, const int32_t *kv_len,
+                    int nthreads)
+{
+    const int fp64 = qd && kd && vd && dod, bits = qb && kb && vb && dob;
+    if (fp64 == bits || !dq || !dk || !dv) return ORACLE_EINVAL;
+    int rc = check_args(B, H, N, d, scale, causal);
+    if (rc) return rc;
+    if (B == 0 || H == 0 || N == 0) return ORACLE_OK;
+    if (Hkv <= 0 || Hkv > H || H % Hkv != 0) return ORACLE_EINVAL;
+    const int G = H / Hkv;
+    const size_t head = (size_t)N * d;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int err = ORACLE_OK;
+    /* one (batch, K/V head) group per iteration: its dK, dV sums stay private */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int g = 0; g < B * Hkv; ++g) {
+        const int b = g / Hkv, hk = g % Hkv;
+        int kv_lim = N;
+        if (kv_len) {
+            kv_lim = kv_len[b];
+            if (kv_lim < 0) kv_lim = 0;
+            if (kv_lim > N) kv_lim = N;
+        }
+        double *buf = (double *)malloc((4 * head + 2 * (size_t)N) * sizeof(double));
+        if (!buf) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+            continue;
+        }
+        double *K = buf, *V = buf + head, *Q = buf + 2 * head, *dO = buf + 3 * head;
+        double *prow = buf + 4 * head, *dsrow = prow + N;
+        const size_t kvbase = (size_t)g * head;
+        for (size_t e = 0; e < head; ++e) {
+            K[e] = bits ? bf16_to_f64(kb[kvbase + e]) : kd[kvbase + e];
+            V[e] = bits ? bf16_to_f64(vb[kvbase + e]) : vd[kvbase + e];
+        }
+        double *dK = dk + kvbase, *dV = dv + kvbase;
+        for (size_t e = 0; e < head; ++e) dK[e] = dV[e] = 0.0;
+        for (int hq = hk * G; hq < (hk + 1) * G; ++hq) {
+            const size_t qbase = ((size_t)b * H + hq) * head;
+            for (size_t e = 0; e < head; ++e) {
+                Q[e] = bits ? bf16_to_f64(qb[qbase + e]) : qd[qbase + e];
+                dO[e] = bits ? bf16_to_f64(dob[qbase + e]) : dod[qbase + e];
+            }
+            for (int i = 0; i < N; ++i)
+                bwd_one_row(Q + (size_t)i * d, dO + (size_t)i * d, K, V, N, d, scale, i, causal,
+                            kv_lim, prow, dsrow, dq + qbase + (size_t)i * d, dK, dV);
+        }
+        free(buf);
+    }
+    return err;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP
