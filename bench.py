@@ -2,7 +2,7 @@
 """Benchmark of the fused attention forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 5] [--decode 1]
+                    [--workload 5] [--decode 1] [--backward]
 
 A step is one full forward (one kernel launch) over the workload's tensors,
 which are resident in device memory before the timed region starts. The
@@ -19,6 +19,7 @@ only a barrier and a max-reduction of the timings ("scaling": "weak").
 bounded row sample of the same workload, in the same unit; under torchrun only
 rank 0 runs it.
 
+--backward times the backward pass (fa_bwd) on the workload's shape instead.
 --decode 1 times the split-KV path instead (one query row per head against an
 8K-key cache with grouped K/V heads), in GB/s of algorithmic bytes.
 """
@@ -563,6 +564,158 @@ def decode_arm(args, w):
     return 0
 
 
+def backward_arm(args, w):
+    """Backward pass: one fa_bwd call per step (the row-statistics kernel, the
+    dK/dV pass and the dQ pass) on the workload's shape, with O and lse from
+    this library's forward and dO ~ N(0,1) resident in HBM. Metric: the
+    backward's algorithmic FLOPs, 2.5 x the forward's (five N x N x d products:
+    S, dP, dV, dK, dQ), per second; the dQ pass recomputes S and dP, so the
+    tensor cores do 7/5 of that count. Replicas only under torchrun."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import io_aware_exact_18_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.load_library()
+    H_kv = w.kv_heads
+    q, k, v, do, _ = workloads.make_bwd_inputs(w.B, w.H, H_kv, w.N, w.d,
+                                               seed=w.index + 100 + 1000 * rank,
+                                               q_mult=w.q_mult)
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    o, lse = fa.attention(qd, kd, vd, scale=w.scale, causal=w.causal)
+    dq, dk, dv = (torch.empty_like(x) for x in (qd, kd, vd))
+    ws_bytes = fa.fa_bwd_workspace_bytes(w.B, w.H, w.N)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+
+    def step():
+        st = fa.fa_bwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(),
+                       lse.data_ptr(), dod.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                       dv.data_ptr(), w.B, w.H, H_kv, w.N, w.d, w.scale, int(w.causal), None,
+                       ws.data_ptr(), ws_bytes, sh)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_bwd")
+
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    st = fa.fa_last_device_error(sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed region")
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    flops = 2.5 * w.flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    # end to end: q, k, v, o, lse, dO copied in from pinned host memory, the
+    # call, the three gradients read back
+    e2e_steps = max(1, min(args.steps, 5))
+    hin = [x.pin_memory() for x in (q, k, v, o.cpu(), lse.cpu(), do)]
+    dins = [qd, kd, vd, o, lse, dod]
+    hout = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (dq, dk, dv)]
+    h2d = sum(x.numel() * x.element_size() for x in hin)
+    d2h = sum(x.numel() * x.element_size() for x in hout)
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for dd_, hh in zip(dins, hin):
+                dd_.copy_(hh, non_blocking=True)
+            fa.attention_bwd(qd, kd, vd, o, lse, dod, scale=w.scale, causal=w.causal, dq=dq,
+                             dk=dk, dv=dv, workspace=ws, stream=sh)
+            for hh, dd_ in zip(hout, (dq, dk, dv)):
+                hh.copy_(dd_, non_blocking=True)
+
+    e2e_step()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_local * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+                "tensor_work_frac": achieved * 7 / 5 / peak,
+                "timed": "whole step: row statistics + dK/dV pass + dQ pass",
+                "kernel": f"fa_bwd_prep<{w.d}> + fa_bwd_dkdv<{w.d}> + fa_bwd_dq<{w.d}>"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nthreads = os.cpu_count() or 1
+        Hs, Ns = min(w.H, 16), min(w.N, 2048)
+        qs, ks, vs, dos, _ = workloads.make_bwd_inputs(1, Hs, Hs, Ns, w.d, seed=3)
+        t = time.perf_counter()
+        oracle.attention_bwd(qs, ks, vs, dos, w.scale, causal=w.causal, nthreads=nthreads)
+        dt = time.perf_counter() - t
+        sflops = 10.0 * Hs * Ns * Ns * w.d * (0.5 if w.causal else 1.0)
+        cpu = {"value": sflops / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+               "sample": f"the same computation at B=1, H={Hs}, N={Ns}, d={w.d} "
+                         f"({'causal' if w.causal else 'full'}), fp64, {nthreads} threads",
+               "seconds": dt}
+    if rank == 0:
+        line = {
+            "metric": "attention bwd TFLOP/s (2.5 x forward FLOPs: 10·B·H·N²·d, half causal)",
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**w.describe(), "pass": "backward", "parallelism": f"replicas x{world}",
+                       "l2": "no flush: Q, K, V, O, dO ({:.0f} MiB each) exceed the 126 MB L2"
+                       .format(w.B * w.H * w.N * w.d * 2 / 2**20)},
+            "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": 3 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -576,6 +729,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (fa_bwd) on the workload instead")
     ap.add_argument("--decode", default=None,
                     help="time the split-KV decode path on this decode workload "
                          "(name, or 1 for the first) instead of square attention")
@@ -600,6 +755,13 @@ def main(argv=None):
                                0, B, H, N, d, causal, H_kv=H_kv)
     else:
         w = workloads.get(args.workload)
+    if args.backward:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the backward line has no reference arm; its cpu_baseline key "
+                              "times the oracle"}), flush=True)
+            return 0
+        return backward_arm(args, w)
     if args.impl == "reference":
         return reference_arm(args, w)
     return our_arm(args, w)

@@ -142,6 +142,36 @@ size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits);
  */
 int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
 
+/*
+ * Backward pass: gradients of the attention of fa_fwd / fa_fwd_gqa for a
+ * scalar loss, given dO = dL/dO. The pages report the training speed-ups of
+ * the method ("FlashAttention (UR)", section "Experimental results") but state
+ * no backward algorithm; this is the exact gradient of the forward definition
+ * (chain rule through the row softmax), with P recomputed tile by tile from Q,
+ * K and the forward's lse (the O(N) statistic of section "Complexity and
+ * optimality"), never stored:
+ *   dV = P^T dO,  dS = P * (dO V^T - D),  D_i = dO_i . O_i,
+ *   dQ = scale dS K,  dK = scale dS^T Q.
+ *   q, o, d_o: bf16 [B, H, N, d]; k, v: bf16 [B, H_kv, N, d] (as fa_fwd_gqa);
+ *   lse: fp32 [B, H, N], the forward's (natural log, scale included);
+ *   dq: bf16 [B, H, N, d] out; dk, dv: bf16 [B, H_kv, N, d] out (a shared K/V
+ *   head gets the sum over its group of query heads);
+ *   causal, kv_len, scale: as in the forward call that produced o and lse.
+ *   d must be 64 or 128 (FA_ERR_UNSUPPORTED otherwise).
+ *   workspace: device memory owned by the caller, 16-byte aligned, at least
+ *   fa_bwd_workspace_bytes(B, H, N) bytes, overlapping no other argument; no
+ *   initialisation needed; scratch after the call.
+ * All outputs are fully written; they must not overlap each other, the inputs
+ * or the workspace. Deterministic (no atomics). Errors as in fa_fwd.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *d_o, void *dq, void *dk, void *dv, int B, int H, int H_kv, int N,
+           int d, float scale, int causal, const int32_t *kv_len, void *workspace,
+           size_t workspace_bytes, void *stream);
+
+/* Workspace bytes of fa_bwd: 2 * B * H * ceil(N / 128) * 128 * 4 (0 if invalid). */
+size_t fa_bwd_workspace_bytes(int B, int H, int N);
+
 /* Bytes of split-KV scratch the library itself holds on each device. */
 #define FA_STATIC_SCRATCH_BYTES (16u << 20)
 

@@ -64,6 +64,11 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd_splitkv_static.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i,
                                           vp]
     lib.fa_fwd_splitkv_static.restype = i
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp,
+                           sz, vp]
+    lib.fa_bwd.restype = i
+    lib.fa_bwd_workspace_bytes.argtypes = [i, i, i]
+    lib.fa_bwd_workspace_bytes.restype = sz
     lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.fa_splitkv_workspace_bytes.restype = sz
     lib.fa_splitkv_default_splits.argtypes = [i, i, i, i, i, i]
@@ -131,6 +136,17 @@ def fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits) -> int:
 
 def fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d) -> int:
     return int(load_library().fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d))
+
+
+def fa_bwd(q, k, v, o, lse, d_o, dq, dk, dv, B, H, H_kv, N, d, scale, causal, kv_len,
+           workspace, workspace_bytes, stream) -> int:
+    """C ABI fa_bwd: dq, dk, dv of the forward for the output gradient d_o."""
+    return load_library().fa_bwd(q, k, v, o, lse, d_o, dq, dk, dv, B, H, H_kv, N, d, scale,
+                                 causal, kv_len, workspace, workspace_bytes, stream)
+
+
+def fa_bwd_workspace_bytes(B, H, N) -> int:
+    return int(load_library().fa_bwd_workspace_bytes(B, H, N))
 
 
 def fa_status_string(status: int) -> str:
@@ -242,3 +258,39 @@ def decode_attention(q, k, v, scale=None, causal=False, kv_len=None, num_splits=
     if check and st != FA_OK:
         raise FAError(st, "fa_fwd_splitkv")
     return out, lse
+
+
+def attention_bwd(q, k, v, o, lse, d_o, scale=None, causal=False, kv_len=None, dq=None,
+                  dk=None, dv=None, workspace=None, stream=None, check=True):
+    """dq, dk, dv for bf16 CUDA tensors of a forward call attention(q, k, v)
+    that returned o and lse, and the output gradient d_o (bf16, like o).
+    Allocates the gradients and the workspace with torch unless given."""
+    import torch
+    for t in (q, k, v, o, d_o):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, o, d_o must be contiguous bf16 CUDA tensors")
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor")
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    if k.shape != (B, H_kv, N, d) or v.shape != k.shape or o.shape != q.shape or \
+            d_o.shape != q.shape or lse.shape != (B, H, N):
+        raise ValueError("shapes of q, k, v, o, lse, d_o do not match")
+    if kv_len is not None and (kv_len.dtype != torch.int32 or not kv_len.is_cuda
+                               or kv_len.shape != (B,)):
+        raise ValueError("kv_len must be a CUDA int32 tensor of shape [B]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = fa_bwd_workspace_bytes(B, H, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device).cuda_stream
+    st = fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk),
+                _ptr(dv), B, H, H_kv, N, d, float(scale), int(bool(causal)), _ptr(kv_len),
+                _ptr(workspace), workspace.numel() * workspace.element_size(), s)
+    if check and st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_combine_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
@@ -52,6 +53,15 @@ struct DeviceState {
     bool supported = false;
     uint32_t* err_ptr = nullptr;
 };
+
+// Opt in to the dynamic shared memory of the two backward passes.
+template <int D>
+bool set_bwd_smem() {
+    return cudaFuncSetAttribute(fa_bwd_dkdv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                BwdCfg<D>::kSmemBytes) == cudaSuccess &&
+           cudaFuncSetAttribute(fa_bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                BwdCfg<D>::kSmemBytes) == cudaSuccess;
+}
 
 // Opt in to the dynamic shared memory of one kernel instantiation.
 template <int D, int QT, bool kGen>
@@ -97,7 +107,8 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
             st.err_ptr = static_cast<uint32_t*>(p);
             const bool ok = set_smem<64, 2, false>() && set_smem<128, 2, false>() &&
                             set_smem<256, 1, false>() && set_smem<64, 1, true>() &&
-                            set_smem<128, 1, true>() && set_smem<256, 1, true>();
+                            set_smem<128, 1, true>() && set_smem<256, 1, true>() &&
+                            set_bwd_smem<64>() && set_bwd_smem<128>();
             if (!ok) return FA_ERR_LAUNCH;
         }
         st.probed = true;
@@ -322,6 +333,95 @@ int static_scratch(void** out) {
     return FA_OK;
 }
 
+// ------------------------------------------------------------------ backward
+// Workspace of the backward pass: lse * log2(e), then D = rowsum(dO * O), each
+// fp32 [B*H][Np] with Np = N rounded up to whole 128-row tiles.
+int64_t bwd_np(int N) { return ((int64_t)N + 127) / 128 * 128; }
+size_t bwd_ws_bytes(int64_t BH, int N) { return 2 * (size_t)BH * (size_t)bwd_np(N) * 4; }
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* d_o, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+             int d, float scale, int causal, const int32_t* kv_len, void* ws, size_t ws_bytes,
+             void* stream) {
+    if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+    if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0 || N == 0) return FA_OK;
+    if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv || !ws)
+        return FA_ERR_INVALID_ARG;
+    const uintptr_t a16 =
+        reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o) |
+        reinterpret_cast<uintptr_t>(d_o) | reinterpret_cast<uintptr_t>(dq) |
+        reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv) |
+        reinterpret_cast<uintptr_t>(ws);
+    if ((a16 & 15u) != 0 || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0)
+        return FA_ERR_INVALID_ARG;
+    const int64_t BH = (int64_t)B * H, BHkv = (int64_t)B * H_kv;
+    const int64_t Np = bwd_np(N), n_t = Np / 128;
+    if (BH * Np > INT32_MAX || BH * n_t > INT32_MAX) return FA_ERR_INVALID_ARG;
+    if (ws_bytes < bwd_ws_bytes(BH, N)) return FA_ERR_INVALID_ARG;
+    const size_t qb = (size_t)BH * N * d * 2, kb = (size_t)BHkv * N * d * 2;
+    const size_t lb = (size_t)BH * N * 4, wb = bwd_ws_bytes(BH, N);
+    struct Buf { const void* p; size_t n; };
+    const Buf outs[4] = {{dq, qb}, {dk, kb}, {dv, kb}, {ws, wb}};
+    const Buf all[10] = {{q, qb}, {k, kb}, {v, kb}, {o, qb}, {lse, lb}, {d_o, qb},
+                         {dq, qb}, {dk, kb}, {dv, kb}, {ws, wb}};
+    for (int a = 0; a < 4; ++a)       // every output against every other buffer
+        for (int c = 0; c < 10; ++c)
+            if (c != 6 + a && overlaps(outs[a].p, outs[a].n, all[c].p, all[c].n))
+                return FA_ERR_INVALID_ARG;
+
+    int dev = 0;
+    uint32_t* err = nullptr;
+    int rc = prepare_device(&dev, &err);
+    if (rc != FA_OK) return rc;
+    alignas(64) CUtensorMap mq, mk, mv, mdo;
+    if ((rc = make_map(&mq, q, (int)BH, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, k, (int)BHkv, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, v, (int)BHkv, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mdo, d_o, (int)BH, N, d)) != FA_OK) return rc;
+
+    float* lse2 = static_cast<float*>(ws);
+    float* dvec = lse2 + BH * Np;
+    BwdParams p{};
+    p.dq = static_cast<__nv_bfloat16*>(dq);
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.lse2 = lse2;
+    p.dvec = dvec;
+    p.kv_len = kv_len;
+    p.dev_err = err;
+    p.B = B;
+    p.H = H;
+    p.H_kv = H_kv;
+    p.N = N;
+    p.Np = (int)Np;
+    p.causal = causal;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.watchdog_ns = kWatchdogNs;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 pgrid((unsigned)((BH * Np + 7) / 8)), pblock(256);
+    const dim3 agrid((unsigned)(BHkv * n_t)), bgrid((unsigned)(BH * n_t)), block(kBwdThreads);
+    const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
+    const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(d_o);
+    if (d == 128) {
+        fa_bwd_prep<128><<<pgrid, pblock, 0, s>>>(ob, dob, lse, lse2, dvec, BH, N, (int)Np);
+        fa_bwd_dkdv<128><<<agrid, block, BwdCfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+        fa_bwd_dq<128><<<bgrid, block, BwdCfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+    } else {
+        fa_bwd_prep<64><<<pgrid, pblock, 0, s>>>(ob, dob, lse, lse2, dvec, BH, N, (int)Np);
+        fa_bwd_dkdv<64><<<agrid, block, BwdCfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+        fa_bwd_dq<64><<<bgrid, block, BwdCfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+    }
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 FwdCall square_call(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int H, int H_kv, int N, int d, float scale, int causal,
                     const int32_t* kv_len) {
@@ -432,6 +532,20 @@ FA_EXPORT int fa_fwd_splitkv_static(const void* q, const void* k, const void* v,
     a.ws = scratch;
     a.ws_bytes = (size_t)FA_STATIC_SCRATCH_BYTES;
     return fa::fwd_impl(a, stream);
+}
+
+FA_EXPORT size_t fa_bwd_workspace_bytes(int B, int H, int N) {
+    if (B < 0 || H < 0 || N < 0) return 0;
+    return fa::bwd_ws_bytes((int64_t)B * H, N);
+}
+
+FA_EXPORT int fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* d_o, void* dq, void* dk, void* dv, int B,
+                     int H, int H_kv, int N, int d, float scale, int causal,
+                     const int32_t* kv_len, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+    return fa::bwd_impl(q, k, v, o, lse, d_o, dq, dk, dv, B, H, H_kv, N, d, scale, causal,
+                        kv_len, workspace, workspace_bytes, stream);
 }
 
 FA_EXPORT const char* fa_status_string(int status) {

@@ -17,7 +17,8 @@ def lib():
 
 
 def test_header_declares_the_boundary():
-    assert fa.declared_symbols() == ["fa_fwd", "fa_fwd_gqa", "fa_fwd_kvlen",
+    assert fa.declared_symbols() == ["fa_bwd", "fa_bwd_workspace_bytes",
+                                     "fa_fwd", "fa_fwd_gqa", "fa_fwd_kvlen",
                                      "fa_fwd_splitkv", "fa_fwd_splitkv_static",
                                      "fa_last_device_error",
                                      "fa_splitkv_default_splits",
@@ -173,3 +174,45 @@ def test_splitkv_default_splits_in_range(lib):
         s = lib.fa_splitkv_default_splits(*args)
         assert 1 <= s <= 128, (args, s)
     assert lib.fa_splitkv_default_splits(0, 32, 8, 1, 8192, 128) == 1
+
+
+# ---------------------------------------------------------------- backward
+BW = dict(q=P, k=P + (1 << 30), v=P + (2 << 30), o=P + (3 << 30), lse=P + (4 << 30),
+          do=P + (5 << 30), dq=P + (6 << 30), dk=P + (7 << 30), dv=P + (8 << 30),
+          B=2, H=8, H_kv=2, N=300, d=128, scale=0.088, causal=1, kv_len=None,
+          ws=P + (9 << 30), ws_bytes=1 << 30)
+
+
+def call_bwd(lib, **over):
+    a = dict(BW, **over)
+    return lib.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"],
+                      a["dv"], a["B"], a["H"], a["H_kv"], a["N"], a["d"], a["scale"],
+                      a["causal"], a["kv_len"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(N=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(H_kv=3), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=2), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=0), fa.FA_ERR_INVALID_ARG),
+    (dict(ws_bytes=1000), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=P + (9 << 30) + 4), fa.FA_ERR_INVALID_ARG),   # misaligned
+    (dict(dq=P), fa.FA_ERR_INVALID_ARG),                   # dq is q
+    (dict(dk=P + (8 << 30)), fa.FA_ERR_INVALID_ARG),       # dk is dv
+    (dict(dv=P + (5 << 30) + 64), fa.FA_ERR_INVALID_ARG),  # dv inside d_o
+    (dict(ws=P + (6 << 30)), fa.FA_ERR_INVALID_ARG),       # workspace is dq
+    (dict(lse=P + (4 << 30) + 2), fa.FA_ERR_INVALID_ARG),
+    (dict(N=0), fa.FA_OK),
+    (dict(B=0, q=0, k=0, v=0, o=0, lse=0, do=0, dq=0, dk=0, dv=0, ws=0), fa.FA_OK),
+])
+def test_bwd_argument_errors_are_synchronous(lib, over, status):
+    assert call_bwd(lib, **over) == status
+
+
+def test_bwd_workspace_bytes(lib):
+    assert lib.fa_bwd_workspace_bytes(2, 8, 300) == 2 * 2 * 8 * 384 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 128) == 2 * 128 * 4
+    assert lib.fa_bwd_workspace_bytes(-1, 1, 1) == 0

@@ -180,6 +180,24 @@ def make_qkv(B, H, H_kv, Nq, Nk, d, seed, kv_len_range=None):
     return q, k, v, kv_len
 
 
+def make_bwd_inputs(B, H, H_kv, N, d, seed, kv_len_range=None, q_mult=1.0):
+    """Inputs of a backward pass: q [B,H,N,d], k, v [B,H_kv,N,d], then the
+    output gradient dO [B,H,N,d] (N(0,1), rounded to bf16), then kv_len."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn((B, H, N, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn((B, H_kv, N, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn((B, H_kv, N, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    do = torch.randn((B, H, N, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    if q_mult != 1.0:
+        q = q * q_mult
+    kv_len = None
+    if kv_len_range is not None:
+        lo, hi = kv_len_range
+        kv_len = torch.randint(lo, hi + 1, (B,), generator=g).to(torch.int32)
+    return q, k, v, do, kv_len
+
+
 def sample_rows(N: int, seed: int, n_random: int = 256, edge: int = 128):
     """Row indices for sampled checks at full size: the first and last `edge`
     rows plus `n_random` seeded random rows, sorted and unique."""
