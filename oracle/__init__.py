@@ -146,8 +146,6 @@ def attention(q, k, v, scale, causal=False, kv_len=None, rows=None,
     u16p = ctypes.POINTER(ctypes.c_uint16)
     rp = None
     if rows is not None:
-        if not qb16:
-            raise ValueError("row subsets are supported for bf16 inputs only")
         ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
         rp = ra.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
     if qb16:
