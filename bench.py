@@ -2,7 +2,7 @@
 """Benchmark of the fused attention forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 5] [--decode 1] [--backward]
+                    [--workload 5] [--decode 1] [--backward] [--fp8]
 
 A step is one full forward (one kernel launch) over the workload's tensors,
 which are resident in device memory before the timed region starts. The
@@ -20,6 +20,7 @@ bounded row sample of the same workload, in the same unit; under torchrun only
 rank 0 runs it.
 
 --backward times the backward pass (fa_bwd) on the workload's shape instead.
+--fp8 times the e4m3 forward (fa_fwd_fp8) on the workload's shape instead.
 --decode 1 times the split-KV path instead (one query row per head against an
 8K-key cache with grouped K/V heads), in GB/s of algorithmic bytes.
 """
@@ -716,6 +717,145 @@ def backward_arm(args, w):
     return 0
 
 
+def fp8_arm(args, w):
+    """The e4m3 forward (fa_fwd_fp8) on the workload's shape: Q, K, V quantized
+    per tensor to e4m3 (descale amax / 448) and resident in HBM, one launch per
+    step. Same metric as the bf16 line (4*B*H*N^2*d, half causal); the roofline
+    peak is the measured bf16 figure times the nominal e4m3 / bf16 ratio (2)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import io_aware_exact_18_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.load_library()
+    q8, k8, v8, sc, _ = workloads.make_fp8_inputs(w.B, w.H, w.kv_heads, w.N, w.d,
+                                                  seed=w.index + 200 + 1000 * rank)
+    qd, kd, vd = (x.to(dev) for x in (q8, k8, v8))
+    od = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    lsed = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+
+    def step():
+        st = fa.fa_fwd_fp8(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), sc[0], sc[1], sc[2],
+                           od.data_ptr(), lsed.data_ptr(), w.B, w.H, w.kv_heads, w.N, w.d,
+                           w.scale, int(w.causal), None, sh)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_fwd_fp8")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    st = fa.fa_last_device_error(sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed region")
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    flops = w.flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    e2e_steps = max(1, min(args.steps, 10))
+    hin = [x.view(torch.uint8).pin_memory() for x in (q8, k8, v8)]
+    din = [x.view(torch.uint8) for x in (qd, kd, vd)]
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    lh = torch.empty(lsed.shape, dtype=lsed.dtype).pin_memory()
+    h2d = sum(x.numel() for x in hin)
+    d2h = oh.numel() * 2 + lh.numel() * 4
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for dd_, hh in zip(din, hin):
+                dd_.copy_(hh, non_blocking=True)
+            fa.attention_fp8(qd, kd, vd, *sc, scale=w.scale, causal=w.causal, out=od, lse=lsed,
+                             stream=sh)
+            oh.copy_(od, non_blocking=True)
+            lh.copy_(lsed, non_blocking=True)
+
+    e2e_step()
+    stream.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_local * 1e-3) / 1e12
+    peak = 2.0 * float(peaks["bf16_tflops"])
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16 burst (cuBLAS) x nominal e4m3/bf16 ratio 2",
+                "kernel": f"fa_fwd_sm100<{w.d},2,square,e4m3>"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import fp8 as ofp8
+        nthreads = os.cpu_count() or 1
+        rows = workloads.sample_rows(w.N, seed=9, n_random=24, edge=4)
+        t = time.perf_counter()
+        ofp8.attention_fp8(q8, k8, v8, *sc, w.scale, causal=w.causal, rows=rows,
+                           nthreads=nthreads)
+        dt = time.perf_counter() - t
+        fl = sum(4.0 * w.d * ((i + 1) if w.causal else w.N) for i in rows) * w.B * w.H
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+               "sample": f"{len(rows)} query rows x all {w.B * w.H} heads of the same e4m3 "
+                         f"inputs, dequantized, fp64, {nthreads} threads", "seconds": dt}
+    if rank == 0:
+        line = {
+            "metric": METRIC + " (e4m3 inputs)", "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3", "data": "synthetic",
+            "config": {**w.describe(), "inputs": "e4m3, per-tensor descale amax/448",
+                       "parallelism": f"replicas x{world}",
+                       "l2": "no flush: inputs (3 x {:.0f} MiB) exceed the 126 MB L2".format(
+                           w.B * w.H * w.N * w.d / 2**20)},
+            "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -729,6 +869,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the e4m3 forward (fa_fwd_fp8) on the workload instead")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (fa_bwd) on the workload instead")
     ap.add_argument("--decode", default=None,
@@ -755,6 +897,13 @@ def main(argv=None):
                                0, B, H, N, d, causal, H_kv=H_kv)
     else:
         w = workloads.get(args.workload)
+    if args.fp8:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the e4m3 line has no reference arm; its cpu_baseline key "
+                              "times the oracle"}), flush=True)
+            return 0
+        return fp8_arm(args, w)
     if args.backward:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable":

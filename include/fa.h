@@ -143,6 +143,25 @@ size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits);
 int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
 
 /*
+ * FP8 forward: q, k, v hold e4m3 codes (OCP 8-bit float: 1 sign, 4 exponent
+ * bits with bias 7, 3 mantissa bits, largest finite 448), one byte each, laid
+ * out like the bf16 tensors of fa_fwd_gqa ([B, H, N, d] and [B, H_kv, N, d]);
+ * q_descale, k_descale, v_descale (finite, > 0) give the tensors' values as
+ * descale * code. The result is the attention of those dequantized tensors,
+ * O bf16 [B, H, N, d] and lse fp32 [B, H, N] as in fa_fwd. This is the
+ * lower-precision-input direction of FlashAttention-3 ("FlashAttention (UR)",
+ * section "FlashAttention-3"): both tile products run on the tensor cores in
+ * e4m3 with fp32 accumulation, and the probabilities P are rounded to e4m3
+ * (relative error up to 2^-4) before the P.V product, so O carries that
+ * error; lse does not (scores are exact products of e4m3 values). d must be
+ * 128 (else FA_ERR_UNSUPPORTED); causal, kv_len, H_kv, errors as in
+ * fa_fwd_gqa.
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, float q_descale, float k_descale,
+               float v_descale, void *o, float *lse, int B, int H, int H_kv, int N, int d,
+               float scale, int causal, const int32_t *kv_len, void *stream);
+
+/*
  * Backward pass: gradients of the attention of fa_fwd / fa_fwd_gqa for a
  * scalar loss, given dO = dL/dO. The pages report the training speed-ups of
  * the method ("FlashAttention (UR)", section "Experimental results") but state

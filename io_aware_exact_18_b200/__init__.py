@@ -64,6 +64,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd_splitkv_static.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i,
                                           vp]
     lib.fa_fwd_splitkv_static.restype = i
+    lib.fa_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, i, vp, vp]
+    lib.fa_fwd_fp8.restype = i
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp,
                            sz, vp]
     lib.fa_bwd.restype = i
@@ -136,6 +138,13 @@ def fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits) -> int:
 
 def fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d) -> int:
     return int(load_library().fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d))
+
+
+def fa_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, B, H, H_kv, N, d, scale,
+               causal, kv_len, stream) -> int:
+    """C ABI fa_fwd_fp8: e4m3 q, k, v with per-tensor descales; bf16 O, fp32 lse."""
+    return load_library().fa_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, B, H,
+                                     H_kv, N, d, scale, causal, kv_len, stream)
 
 
 def fa_bwd(q, k, v, o, lse, d_o, dq, dk, dv, B, H, H_kv, N, d, scale, causal, kv_len,
@@ -294,3 +303,31 @@ def attention_bwd(q, k, v, o, lse, d_o, scale=None, causal=False, kv_len=None, d
     if check and st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def attention_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal=False,
+                  kv_len=None, out=None, lse=None, stream=None, check=True):
+    """O (bf16), lse for e4m3 CUDA tensors (torch.float8_e4m3fn or uint8 codes)
+    q8 [B, H, N, d] and k8, v8 [B, H_kv, N, d] with per-tensor descales,
+    through fa_fwd_fp8."""
+    import torch
+    for t in (q8, k8, v8):
+        if t.element_size() != 1 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q8, k8, v8 must be contiguous one-byte CUDA tensors")
+    B, H, N, d = q8.shape
+    H_kv = k8.shape[1]
+    if k8.shape != (B, H_kv, N, d) or v8.shape != k8.shape:
+        raise ValueError(f"bad shapes {q8.shape} {k8.shape} {v8.shape}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    s = stream if stream is not None else torch.cuda.current_stream(q8.device).cuda_stream
+    st = fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_descale), float(k_descale),
+                    float(v_descale), _ptr(out), _ptr(lse), B, H, H_kv, N, d, float(scale),
+                    int(bool(causal)), _ptr(kv_len), s)
+    if check and st != FA_OK:
+        raise FAError(st, "fa_fwd_fp8")
+    return out, lse

@@ -64,11 +64,11 @@ bool set_bwd_smem() {
 }
 
 // Opt in to the dynamic shared memory of one kernel instantiation.
-template <int D, int QT, bool kGen>
+template <int D, int QT, bool kGen, int E = 2>
 bool set_smem() {
-    return cudaFuncSetAttribute(fa_fwd_sm100<D, QT, kGen>,
+    return cudaFuncSetAttribute(fa_fwd_sm100<D, QT, kGen, E>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Cfg<D, QT>::kSmemBytes) == cudaSuccess;
+                                Cfg<D, QT, E>::kSmemBytes) == cudaSuccess;
 }
 
 std::mutex g_mutex;
@@ -108,7 +108,8 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
             const bool ok = set_smem<64, 2, false>() && set_smem<128, 2, false>() &&
                             set_smem<256, 1, false>() && set_smem<64, 1, true>() &&
                             set_smem<128, 1, true>() && set_smem<256, 1, true>() &&
-                            set_bwd_smem<64>() && set_bwd_smem<128>();
+                            set_smem<128, 2, false, 1>() && set_bwd_smem<64>() &&
+                            set_bwd_smem<128>();
             if (!ok) return FA_ERR_LAUNCH;
         }
         st.probed = true;
@@ -119,19 +120,20 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
     return FA_OK;
 }
 
-// 3-D view [B*H, N, d] of a contiguous bf16 tensor; box = 64 columns (128
-// bytes, the swizzle width) x box_rows rows x box_planes heads. The third
-// dimension keeps a tile from ever crossing into the next head: rows past N
-// read as zero.
+// 3-D view [B*H, N, d] of a contiguous bf16 (elem = 2) or 8-bit (elem = 1)
+// tensor; box = 128 bytes of columns (the swizzle width) x box_rows rows x
+// box_planes heads. The third dimension keeps a tile from ever crossing into
+// the next head: rows past N read as zero.
 int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows = 128,
-             int box_planes = 1) {
+             int box_planes = 1, int elem = 2) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return FA_ERR_LAUNCH;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_planes};
+    cuuint64_t strides[2] = {(cuuint64_t)d * elem, (cuuint64_t)N * (cuuint64_t)d * elem};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / elem), (cuuint32_t)box_rows, (cuuint32_t)box_planes};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+    CUresult r = enc(map, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                     3, const_cast<void*>(ptr), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -157,6 +159,8 @@ struct FwdCall {
     bool pack;           // pack the query heads of a K/V group into one tile
     void* ws;            // split partials (splits > 1)
     size_t ws_bytes;
+    int elem = 2;        // bytes per element of q, k, v: 2 (bf16) or 1 (e4m3)
+    float q_descale = 1.f, k_descale = 1.f, v_descale = 1.f;   // e4m3 inputs
 };
 
 // Workspace layout for `splits` ranges: O partials fp32 [splits][B*H][Nq][d],
@@ -191,6 +195,12 @@ int fwd_impl(const FwdCall& a, void* stream) {
     if (!std::isfinite(a.scale) || !(a.scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (a.splits < 1 || a.splits > kMaxSplits) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+    const int E = a.elem;
+    if (E == 1) {
+        if (d != 128) return FA_ERR_UNSUPPORTED;
+        for (float x : {a.q_descale, a.k_descale, a.v_descale})
+            if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
+    }
     if (B == 0 || H == 0 || Nq == 0) return FA_OK;
     if (!a.q || !a.k || !a.v || !a.o || !a.lse) return FA_ERR_INVALID_ARG;
     const uintptr_t a16 = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
@@ -205,6 +215,7 @@ int fwd_impl(const FwdCall& a, void* stream) {
     // Square attention (one key range, no packing, Nq == Nk) runs the
     // specialised kernels; everything else the general one-query-tile kernel.
     const bool general = a.splits > 1 || G > 1 || Nq != Nk;
+    if (E == 1 && general) return FA_ERR_UNSUPPORTED;   // e4m3: square attention only
     const int qt = (general || d == 256) ? 1 : 2;          // query tiles per unit
     const int64_t n_rb = ((int64_t)Nq + nq_blk - 1) / nq_blk;
     const int64_t n_units = (n_rb + qt - 1) / qt * a.splits;
@@ -214,9 +225,10 @@ int fwd_impl(const FwdCall& a, void* stream) {
     const int64_t rows = BH * Nq;
     if (rows > INT32_MAX) return FA_ERR_INVALID_ARG;      // row indices are 32-bit in the kernel
     const size_t tbytes = (size_t)rows * d * 2, lbytes = (size_t)rows * 4;
-    const size_t kvbytes = (size_t)BHkv * (size_t)Nk * (size_t)d * 2;
-    if (overlaps(a.o, tbytes, a.q, tbytes) || overlaps(a.o, tbytes, a.k, kvbytes) ||
-        overlaps(a.o, tbytes, a.v, kvbytes) || overlaps(a.lse, lbytes, a.q, tbytes) ||
+    const size_t qbytes = (size_t)rows * d * E;
+    const size_t kvbytes = (size_t)BHkv * (size_t)Nk * (size_t)d * E;
+    if (overlaps(a.o, tbytes, a.q, qbytes) || overlaps(a.o, tbytes, a.k, kvbytes) ||
+        overlaps(a.o, tbytes, a.v, kvbytes) || overlaps(a.lse, lbytes, a.q, qbytes) ||
         overlaps(a.lse, lbytes, a.k, kvbytes) || overlaps(a.lse, lbytes, a.v, kvbytes) ||
         overlaps(a.lse, lbytes, a.o, tbytes))
         return FA_ERR_INVALID_ARG;
@@ -226,7 +238,7 @@ int fwd_impl(const FwdCall& a, void* stream) {
         const size_t need = ws_total_bytes(rows, d, a.splits);
         if (a.ws == nullptr || a.ws_bytes < need || (reinterpret_cast<uintptr_t>(a.ws) & 15u) != 0)
             return FA_ERR_INVALID_ARG;
-        if (overlaps(a.ws, need, a.q, tbytes) || overlaps(a.ws, need, a.k, kvbytes) ||
+        if (overlaps(a.ws, need, a.q, qbytes) || overlaps(a.ws, need, a.k, kvbytes) ||
             overlaps(a.ws, need, a.v, kvbytes) || overlaps(a.ws, need, a.o, tbytes) ||
             overlaps(a.ws, need, a.lse, lbytes))
             return FA_ERR_INVALID_ARG;
@@ -241,9 +253,9 @@ int fwd_impl(const FwdCall& a, void* stream) {
     if (rc != FA_OK) return rc;
 
     alignas(64) CUtensorMap mq, mk, mv;
-    if ((rc = make_map(&mq, a.q, (int)BH, Nq, d, nq_blk, G)) != FA_OK) return rc;
-    if ((rc = make_map(&mk, a.k, (int)BHkv, Nk, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, a.v, (int)BHkv, Nk, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mq, a.q, (int)BH, Nq, d, nq_blk, G, E)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, a.k, (int)BHkv, Nk, d, 128, 1, E)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, a.v, (int)BHkv, Nk, d, 128, 1, E)) != FA_OK) return rc;
 
     FwdParams p{};
     p.o = static_cast<__nv_bfloat16*>(a.o);
@@ -273,11 +285,18 @@ int fwd_impl(const FwdCall& a, void* stream) {
     p.group_heads = (int)((BHB + groups - 1) / groups);
     p.causal = a.causal;
     p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.o_mul = 1.f;
+    if (E == 1) {
+        p.scale_log2 = (float)((double)a.scale * a.q_descale * a.k_descale * 1.4426950408889634);
+        p.o_mul = a.v_descale;
+    }
     p.watchdog_ns = kWatchdogNs;
 
     const dim3 grid((unsigned)(BHB * n_units)), block(kThreads);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (general) {
+    if (E == 1) {
+        fa_fwd_sm100<128, 2, false, 1><<<grid, block, Cfg<128, 2, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+    } else if (general) {
         if (d == 256)
             fa_fwd_sm100<256, 1, true><<<grid, block, Cfg<256, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
         else if (d == 128)
@@ -531,6 +550,18 @@ FA_EXPORT int fa_fwd_splitkv_static(const void* q, const void* k, const void* v,
     if (rc != FA_OK) return rc;
     a.ws = scratch;
     a.ws_bytes = (size_t)FA_STATIC_SCRATCH_BYTES;
+    return fa::fwd_impl(a, stream);
+}
+
+FA_EXPORT int fa_fwd_fp8(const void* q, const void* k, const void* v, float q_descale,
+                         float k_descale, float v_descale, void* o, float* lse, int B, int H,
+                         int H_kv, int N, int d, float scale, int causal,
+                         const int32_t* kv_len, void* stream) {
+    fa::FwdCall a = fa::square_call(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, kv_len);
+    a.elem = 1;
+    a.q_descale = q_descale;
+    a.k_descale = k_descale;
+    a.v_descale = v_descale;
     return fa::fwd_impl(a, stream);
 }
 

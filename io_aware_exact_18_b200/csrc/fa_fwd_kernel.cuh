@@ -94,16 +94,19 @@ constexpr float kLn2 = 0.69314718055994530942f;
 // current ones. d = 256 needs it (O alone takes 256 TMEM columns); the
 // split-KV kernel uses it at every d, since a short query block gives the
 // second tile of a pair nothing to do.
-template <int D, int QT>
+// E is the element size of Q, K and V: 2 (bf16) or 1 (e4m3, d = 128 only).
+template <int D, int QT, int E = 2>
 struct Cfg {
     static_assert(D == 64 || D == 128 || D == 256, "head dim 64, 128 or 256");
     static_assert(QT == 1 || (QT == 2 && D <= 128), "two query tiles need d <= 128");
+    static_assert(E == 2 || (E == 1 && D == 128), "e4m3 inputs need d = 128");
     static constexpr int kQT = QT;                        // query tiles per unit
-    static constexpr int kBlocks = D / 64;                // 128-byte column blocks per row
+    static constexpr int kBlocks = D * E / 128;           // 128-byte column blocks per row
+    static constexpr int kBlockElems = 128 / E;           // columns of one block
     static constexpr int kBlockBytes = kTile * 128;       // 16 KB
-    static constexpr int kTileBytes = kTile * D * 2;      // one Q/K/V tile
+    static constexpr int kTileBytes = kTile * D * E;      // one Q/K/V tile
     static constexpr int kSlots =                         // K/V ring depth
-        (D == 256) ? 2 : (D == 128) ? (QT == 2 ? 4 : 5) : 8;
+        (E == 1) ? 8 : (D == 256) ? 2 : (D == 128) ? (QT == 2 ? 4 : 5) : 8;
     static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 1024 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
@@ -134,7 +137,8 @@ struct FwdParams {
     int n_units;               // units per head block: ceil(n_rb / query tiles per unit) * splits
     int group_heads;           // head blocks per L2 group (launch order)
     int causal;
-    float scale_log2;          // scale * log2(e)
+    float scale_log2;          // scale * log2(e) (times the Q and K descales for e4m3 inputs)
+    float o_mul;               // 1, or the V descale for e4m3 inputs
     uint64_t watchdog_ns;
 };
 
@@ -242,32 +246,59 @@ __device__ __forceinline__ float row_max(const float (&s)[kTile]) {
     return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
 }
 
-// P = exp2(s*c - mc), rounded to bf16 pairs and written over the row's S in
-// TMEM (warp-wide stores); returns the row sum of the fp32 probabilities.
+// P = exp2(s*c - mc), rounded to bf16 pairs (E = 2: 64 TMEM columns) or to
+// e4m3 quadruples (E = 1: 32 columns) and written over the row's S in TMEM
+// (warp-wide stores); returns the row sum of the fp32 probabilities.
+template <int E>
 __device__ __forceinline__ float exp_tile(const float (&s)[kTile], float c, float mc,
                                           uint32_t tS) {
     float sum0 = 0.f, sum1 = 0.f;
+    if constexpr (E == 2) {
 #pragma unroll
-    for (int ch = 0; ch < kTile / 32; ++ch) {
-        uint32_t packed[16];
+        for (int ch = 0; ch < kTile / 32; ++ch) {
+            uint32_t packed[16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
-            const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
-            sum0 += p0;
-            sum1 += p1;
-            packed[q] = pack_bf16x2(p0, p1);
+            for (int q = 0; q < 16; ++q) {
+                const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
+                const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
+                sum0 += p0;
+                sum1 += p1;
+                packed[q] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + (uint32_t)(ch * 16), packed);
         }
-        tmem_st16(tS + (uint32_t)(ch * 16), packed);
+    } else {
+#pragma unroll
+        for (int ch = 0; ch < kTile / 64; ++ch) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                float pq[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pq[e] = fast_exp2(fmaf(s[ch * 64 + 4 * q + e], c, -mc));
+                sum0 += pq[0] + pq[2];
+                sum1 += pq[1] + pq[3];
+                packed[q] = pack_e4m3x4(pq[0], pq[1], pq[2], pq[3]);
+            }
+            tmem_st16(tS + (uint32_t)(ch * 16), packed);
+        }
     }
     return sum0 + sum1;
 }
 
-template <int D, int QT, bool kGen>
+// Largest row sum of a tile's probabilities before the row takes its true
+// maximum: 2^64 for bf16 P; 256 for e4m3 P, whose largest finite value is 448,
+// so every probability of an accepted tile is representable.
+template <int E>
+__device__ __forceinline__ constexpr float max_tile_sum() {
+    return E == 2 ? kMaxTileSum : 256.0f;
+}
+
+template <int D, int QT, bool kGen, int E = 2>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = Cfg<D, QT>;
+    using C = Cfg<D, QT, E>;
     const Shape<kGen> sh(p);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -365,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
                 for (int blk = 0; blk < C::kBlocks; ++blk)
                     tma_load_3d_hint(map, &bars->kv_full[slot], dst + blk * C::kBlockBytes,
-                                     blk * 64, (u.kt0 + tile) * kTile, u.bkv, pol_kv);
+                                     blk * C::kBlockElems, (u.kt0 + tile) * kTile, u.bkv,
+                                     pol_kv);
                 ++L;
                 return true;
             };
@@ -391,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (u.n[t] > 0)
                         for (int blk = 0; blk < C::kBlocks; ++blk)
                             tma_load_3d_hint(&tm_q, &bars->q_full[t], sQ[t] + blk * C::kBlockBytes,
-                                             blk * 64, (u.rb0 + t) * sh.nq_blk,
+                                             blk * C::kBlockElems, (u.rb0 + t) * sh.nq_blk,
                                              u.b * p.H + u.h0, pol_q);
                 }
                 // the rest of K_0, V_0, K_1, V_1, ... of this unit
@@ -423,10 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         // ====================================================== MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTile, 0, 0);
+            constexpr uint32_t idesc_qk = (E == 2) ? idesc_bf16_f32(128, kTile, 0, 0)
+                                                   : idesc_e4m3_f32(128, kTile, 0, 0);
             constexpr int kPvN = (D > 128) ? 128 : D;          // N of one P.V MMA
             constexpr int kPvHalves = D / kPvN;
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kPvN, 0, 1);
+            constexpr uint32_t idesc_pv = (E == 2) ? idesc_bf16_f32(128, kPvN, 0, 1)
+                                                   : idesc_e4m3_f32(128, kPvN, 0, 1);
+            constexpr int kStepRows = 32 / E;                  // keys per 32-byte K-step
             // Descriptors are built once; a tile's start address is added in
             // 16-byte units to the low field (addresses stay below 256 KB).
             const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ[0]), 16, 1024);
@@ -438,10 +473,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t a = dq0 + (uint64_t)t * kTileStep;
                 const uint64_t b = dk0 + (uint64_t)slot * kTileStep;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < D * E / 32; ++kk) {      // 32-byte K-steps
                     const uint64_t off =
                         (uint64_t)(((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4);
-                    umma_ss(tmem + C::col_s(sb), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    if constexpr (E == 2)
+                        umma_ss(tmem + C::col_s(sb), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    else
+                        umma_ss_f8(tmem + C::col_s(sb), a + off, b + off, idesc_qk,
+                                   kk > 0 ? 1u : 0u);
                 }
             };
             // O of tile t (+)= P in S buffer sb . V tile in `slot`. At d = 256 each
@@ -450,13 +489,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue_pv = [&](int t, int sb, int slot, bool accumulate) {
                 const uint64_t b = dv0 + (uint64_t)slot * kTileStep;
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
+                for (int kk = 0; kk < kTile / kStepRows; ++kk) {
 #pragma unroll
                     for (int h = 0; h < kPvHalves; ++h) {
-                        umma_ts(tmem + C::col_o(t) + (uint32_t)(h * kPvN),
-                                tmem + C::col_s(sb) + (uint32_t)(kk * 8),
-                                b + (uint64_t)((kk * 16 * 128 + h * (kPvN / 64) * C::kBlockBytes) >> 4),
-                                idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                        const uint64_t bk = b + (uint64_t)((kk * kStepRows * 128 +
+                                                            h * (kPvN / 64) * C::kBlockBytes) >> 4);
+                        if constexpr (E == 2)
+                            umma_ts(tmem + C::col_o(t) + (uint32_t)(h * kPvN),
+                                    tmem + C::col_s(sb) + (uint32_t)(kk * 8), bk, idesc_pv,
+                                    (accumulate || kk > 0) ? 1u : 0u);
+                        else
+                            umma_ts_f8(tmem + C::col_o(t), tmem + C::col_s(sb) + (uint32_t)(kk * 8),
+                                       bk, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
                     }
                 }
             };
@@ -686,8 +730,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float alpha = 1.f;
                 if (m_ref == -INFINITY) m_ref = row_max(s);
                 float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-                float l_tile = exp_tile(s, c, mc, tS);
-                const bool stale = !(l_tile <= kMaxTileSum);
+                float l_tile = exp_tile<E>(s, c, mc, tS);
+                const bool stale = !(l_tile <= max_tile_sum<E>());
                 if (__any_sync(0xffffffffu, stale)) {
                     if (stale) {
                         const float m_new = fmaxf(m_ref, row_max(s));
@@ -697,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         rescale = true;
                     }
                     mc = m_ref * c;
-                    l_tile = exp_tile(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
+                    l_tile = exp_tile<E>(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
                 }
                 l += l_tile;
                 if (__any_sync(0xffffffffu, rescale)) {
@@ -741,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const bool write = row_id >= 0;
-            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            const float inv_l = (l > 0.f) ? p.o_mul / l : 0.f;
             const float row_lse = (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
             const size_t orow_idx = (size_t)row_id;
             const size_t prow_idx = (size_t)u.s * ((size_t)p.B * p.H * sh.Nq) + (size_t)row_id;

@@ -18,7 +18,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert fa.declared_symbols() == ["fa_bwd", "fa_bwd_workspace_bytes",
-                                     "fa_fwd", "fa_fwd_gqa", "fa_fwd_kvlen",
+                                     "fa_fwd", "fa_fwd_fp8", "fa_fwd_gqa", "fa_fwd_kvlen",
                                      "fa_fwd_splitkv", "fa_fwd_splitkv_static",
                                      "fa_last_device_error",
                                      "fa_splitkv_default_splits",
@@ -216,3 +216,26 @@ def test_bwd_workspace_bytes(lib):
     assert lib.fa_bwd_workspace_bytes(2, 8, 300) == 2 * 2 * 8 * 384 * 4
     assert lib.fa_bwd_workspace_bytes(1, 1, 128) == 2 * 128 * 4
     assert lib.fa_bwd_workspace_bytes(-1, 1, 1) == 0
+
+
+# ---------------------------------------------------------------- e4m3 forward
+@pytest.mark.parametrize("over,status", [
+    (dict(d=64), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(qs=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(ks=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(vs=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(vs=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(H_kv=3), fa.FA_ERR_INVALID_ARG),
+    (dict(o=P), fa.FA_ERR_INVALID_ARG),
+    (dict(N=0), fa.FA_OK),
+])
+def test_fp8_argument_errors_are_synchronous(lib, over, status):
+    a = dict(q=P, k=P + (1 << 30), v=P + (2 << 30), o=P + (3 << 30), lse=P + (4 << 30),
+             qs=0.01, ks=0.01, vs=0.01, B=1, H=8, H_kv=2, N=300, d=128, scale=0.088,
+             causal=1)
+    a.update(over)
+    st = lib.fa_fwd_fp8(a["q"], a["k"], a["v"], a["qs"], a["ks"], a["vs"], a["o"], a["lse"],
+                        a["B"], a["H"], a["H_kv"], a["N"], a["d"], a["scale"], a["causal"],
+                        None, None)
+    assert st == status

@@ -1,0 +1,96 @@
+"""GPU parity of the e4m3 forward (fa_fwd_fp8) against the fp64 oracle on the
+dequantized inputs (oracle.fp8.attention_fp8).
+
+Tolerance, derived from the arithmetic: scores are exact (products of e4m3
+values are exact in fp32; accumulation is fp32), so lse keeps the bf16 path's
+bound |d lse| / max(|lse_ref|, 1) <= 1e-3. Each probability is rounded to
+e4m3 before the P.V product: relative error at most 2^-4 (3 mantissa bits).
+With weights summing to one after normalisation, |dO| <= 2^-4 * max|V|, plus
+bf16 rounding of O (2^-8 * max|O|): that is the element-wise bound. The mean
+error, an average of independent roundings, is bounded by 2^-7 * max|V|.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import fp8 as ofp8
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import io_aware_exact_18_b200 as fa
+    from io_aware_exact_18_b200 import build
+    build.build()
+    fa.load_library()
+    return fa
+
+
+def run_fp8(fa, q8, k8, v8, sc, causal, kv_len=None):
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (x.to(dev) for x in (q8, k8, v8))
+    kvd = None if kv_len is None else kv_len.to(dev)
+    B, H, N, d = q8.shape
+    out = torch.full((B, H, N, d), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
+    fa.attention_fp8(qd, kd, vd, *sc, causal=causal, kv_len=kvd, out=out, lse=lse)
+    st = fa.fa_last_device_error(torch.cuda.current_stream().cuda_stream)
+    assert st == fa.FA_OK, fa.fa_status_string(st)
+    return out.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+def compare_fp8(o, lse, o_ref, lse_ref, vmax, what, rows=None):
+    if rows is not None:
+        o, lse = o[:, :, rows], lse[:, :, rows]
+    assert not np.isnan(o).any() and not np.isnan(lse).any(), f"{what}: unwritten output"
+    dead = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), dead), f"{what}: -inf pattern differs"
+    err = np.abs(o - o_ref)
+    bound = 2.0 ** -4 * vmax + 2.0 ** -8 * np.abs(o_ref).max()
+    assert err.max() <= bound, f"{what}: max|dO| {err.max():.3e} > {bound:.3e}"
+    assert err.mean() <= 2.0 ** -7 * vmax, f"{what}: mean|dO| {err.mean():.3e}"
+    live = ~dead
+    rel = np.abs(lse[live] - lse_ref[live]) / np.maximum(np.abs(lse_ref[live]), 1.0)
+    assert rel.size == 0 or rel.max() <= 1e-3, f"{what}: lse rel err {rel.max():.3e}"
+    return float(err.max() / vmax), float(err.mean() / vmax)
+
+
+def check_fp8(fa, B, H, H_kv, N, causal, seed, kv_len_range=None, rows=None):
+    q8, k8, v8, sc, kvl = workloads.make_fp8_inputs(B, H, H_kv, N, 128, seed, kv_len_range)
+    o, lse = run_fp8(fa, q8, k8, v8, sc, causal, kvl)
+    o_ref, lse_ref = ofp8.attention_fp8(q8, k8, v8, *sc, 1.0 / math.sqrt(128), causal=causal,
+                                        kv_len=kvl, rows=rows)
+    vmax = float(np.abs(ofp8.decode_e4m3(v8.view(torch.uint8).numpy())).max() * sc[2])
+    return compare_fp8(o, lse, o_ref, lse_ref, vmax, f"B{B} H{H}/{H_kv} N{N} c{causal}", rows)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 128, 300, 1024])
+def test_fp8_lengths(fa, N, causal):
+    check_fp8(fa, 2, 2, 2, N, causal, seed=6000 + N + causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_grouped_heads_and_padding(fa, causal):
+    check_fp8(fa, 2, 8, 2, 700, causal, seed=6100 + causal, kv_len_range=(0, 700))
+
+
+def test_fp8_full_size_sampled(fa):
+    """The long-context shape (B1 H32 N16384 causal) in one launch, checked on
+    sampled rows of every head."""
+    N = 16384
+    rows = workloads.sample_rows(N, seed=61, n_random=48, edge=16)
+    check_fp8(fa, 1, 32, 32, N, True, seed=6200, rows=rows)
+
+
+def test_fp8_is_deterministic(fa):
+    q8, k8, v8, sc, _ = workloads.make_fp8_inputs(1, 4, 4, 999, 128, 6300)
+    a = run_fp8(fa, q8, k8, v8, sc, True)
+    b = run_fp8(fa, q8, k8, v8, sc, True)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])

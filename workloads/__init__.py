@@ -198,6 +198,28 @@ def make_bwd_inputs(B, H, H_kv, N, d, seed, kv_len_range=None, q_mult=1.0):
     return q, k, v, do, kv_len
 
 
+def make_fp8_inputs(B, H, H_kv, N, d, seed, kv_len_range=None):
+    """e4m3 inputs: the same draws as make_inputs (Q, then K, then V, N(0,1)
+    fp32), each divided by its descale amax / 448 and rounded to e4m3 by
+    torch's float8_e4m3fn conversion (round to nearest even, no saturation
+    needed). Returns (q8, k8, v8, (q_descale, k_descale, v_descale), kv_len)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    xs = [torch.randn(shape, generator=g, dtype=torch.float32)
+          for shape in ((B, H, N, d), (B, H_kv, N, d), (B, H_kv, N, d))]
+    kv_len = None
+    if kv_len_range is not None:
+        lo, hi = kv_len_range
+        kv_len = torch.randint(lo, hi + 1, (B,), generator=g).to(torch.int32)
+    out, scales = [], []
+    for x in xs:
+        amax = float(x.abs().max()) if x.numel() else 1.0
+        sc = (amax / 448.0) if amax > 0 else 1.0
+        out.append((x / sc).to(torch.float8_e4m3fn))
+        scales.append(sc)
+    return out[0], out[1], out[2], tuple(scales), kv_len
+
+
 def sample_rows(N: int, seed: int, n_random: int = 256, edge: int = 128):
     """Row indices for sampled checks at full size: the first and last `edge`
     rows plus `n_random` seeded random rows, sorted and unique."""
