@@ -92,8 +92,10 @@ struct BwdBarriers {
     uint64_t fixed_full;       // the CTA's two fixed tiles have landed
     uint64_t st_full[4];
     uint64_t st_empty[4];
-    uint64_t s_full;           // S and dP of the current item are in TMEM
-    uint64_t p_full;           // the compute warps have written P / dS (256 arrivals)
+    uint64_t s_full;           // S of the current item is in TMEM
+    uint64_t dp_full;          // dP of the current item is in TMEM
+    uint64_t p_done;           // compute phase 1 done: P written (pass A) / S read (pass B)
+    uint64_t ds_done;          // compute phase 2 done: dS written (256 arrivals each)
     uint64_t acc_done;         // every accumulating MMA has completed
     uint64_t teardown;
     uint32_t tmem_base;
@@ -180,7 +182,9 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdBarriers* bars, const BwdParams
             mbar_init(&bars->st_empty[s], 1);
         }
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, kBwdComputeThreads);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->p_done, kBwdComputeThreads);
+        mbar_init(&bars->ds_done, kBwdComputeThreads);
         mbar_init(&bars->acc_done, 1);
         mbar_init(&bars->teardown, 1);
         bars->abort = 0;
@@ -203,45 +207,65 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdBarriers* bars, const BwdParams
     return bars->tmem_base;
 }
 
-// One thread's half row of a 128 x 128 tile: read columns [c0, c0 + 64) of S
-// and dP (fp32) from TMEM (one wait), form P = exp2(s * c - lse2) on visible
-// entries and dS = P * (dP - D), and write dS (bf16 pairs) to dP's columns
-// [c0, c0 + 32) and, when kWriteP, P to S's columns [c0, c0 + 32).
-// `visible(col)` says whether column col of this thread's row is a visible
-// (query, key) pair; `col_vals(col, l2, dd)` gives lse2 and D of columns
+// The compute warps' work on one 128 x 128 tile, in two phases so the tensor
+// cores can run between them. Each thread owns one row (TMEM lane) and the 64
+// columns [c0, c0 + 64) of it.
+//
+// Phase 1: read S (fp32) and form P = exp2(s * c - lse2) on visible entries
+// (0 elsewhere) into pv; when kWriteP, also write P (bf16 pairs) to S's
+// columns [c0, c0 + 32). `visible(col)` tells whether column col of the row is
+// a visible (query, key) pair; `col_l2(col, l2)` gives lse2 of columns
 // col..col+3 (pass A: per column; pass B: the row's own).
-template <bool kWriteP, typename Vis, typename ColVals>
-__device__ __forceinline__ void bwd_softmax_half(uint32_t tS, uint32_t tDP, int c0, float c,
-                                                 Vis visible, ColVals col_vals) {
-    uint32_t s0[32], s1[32], d0[32], d1[32];
+template <bool kWriteP, typename Vis, typename ColL2>
+__device__ __forceinline__ void bwd_p_half(uint32_t tS, int c0, float c, Vis visible,
+                                           ColL2 col_l2, float (&pv)[64]) {
+    uint32_t s0[32], s1[32];
     tmem_ld32(tS + (uint32_t)c0, s0);
     tmem_ld32(tS + (uint32_t)(c0 + 32), s1);
-    tmem_ld32(tDP + (uint32_t)c0, d0);
-    tmem_ld32(tDP + (uint32_t)(c0 + 32), d1);
     tmem_wait_ld();
-    uint32_t pk[32], dk[32];
 #pragma unroll
     for (int q = 0; q < 64; q += 4) {
-        float l2[4], dd[4];
-        col_vals(c0 + q, l2, dd);
-        float pv[4], dsv[4];
+        float l2[4];
+        col_l2(c0 + q, l2);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int qe = q + e;
             const float sv = __uint_as_float(qe < 32 ? s0[qe] : s1[qe - 32]);
-            const float dpv = __uint_as_float(qe < 32 ? d0[qe] : d1[qe - 32]);
-            const float pe = visible(c0 + qe) ? fast_exp2(fmaf(sv, c, -l2[e])) : 0.f;
-            pv[e] = pe;
-            dsv[e] = pe * (dpv - dd[e]);
+            pv[qe] = visible(c0 + qe) ? fast_exp2(fmaf(sv, c, -l2[e])) : 0.f;
         }
-        pk[q / 2] = pack_bf16x2(pv[0], pv[1]);
-        pk[q / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+    }
+    if (kWriteP) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) pk[q] = pack_bf16x2(pv[2 * q], pv[2 * q + 1]);
+        tmem_st32(tS + (uint32_t)c0, pk);
+    }
+}
+
+// Phase 2: read dP (fp32), form dS = P * (dP - D) and write it (bf16 pairs) to
+// dP's columns [c0, c0 + 32). `col_d(col, dd)` gives D of columns col..col+3.
+template <typename ColD>
+__device__ __forceinline__ void bwd_ds_half(uint32_t tDP, int c0, const float (&pv)[64],
+                                            ColD col_d) {
+    uint32_t d0[32], d1[32];
+    tmem_ld32(tDP + (uint32_t)c0, d0);
+    tmem_ld32(tDP + (uint32_t)(c0 + 32), d1);
+    tmem_wait_ld();
+    uint32_t dk[32];
+#pragma unroll
+    for (int q = 0; q < 64; q += 4) {
+        float dd[4];
+        col_d(c0 + q, dd);
+        float dsv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int qe = q + e;
+            dsv[e] = pv[qe] * (__uint_as_float(qe < 32 ? d0[qe] : d1[qe - 32]) - dd[e]);
+        }
         dk[q / 2] = pack_bf16x2(dsv[0], dsv[1]);
         dk[q / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
     }
-    if (kWriteP) tmem_st32(tS + (uint32_t)c0, pk);
     tmem_st32(tDP + (uint32_t)c0, dk);
-    tmem_wait_st();
 }
 
 // ------------------------------------------------------------------ pass A: dK, dV
@@ -325,23 +349,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t st_k = smem_desc_sw128(smem_u32(sStage), 16, 1024);             // K-major
             const uint64_t st_mn = smem_desc_sw128(smem_u32(sStage), C::kBlockBytes, 1024); // MN-major
             constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
+            // Per item w: S^T(w), dP^T(w) | P(w) -> dV(w), S^T(w+1) | dS(w) -> dK(w),
+            // dP^T(w+1). S^T(w+1) overwrites P(w) after dV(w) has read it, dP^T(w+1)
+            // overwrites dS(w) after dK(w) (tcgen05 MMAs of one thread run in issue
+            // order), so the exponentials of item w+1 overlap dK(w) and dP^T(w+1).
+            auto q_off = [&](int w) { return (uint64_t)(w % C::kStages) * 2 * kTileStep; };
+            auto wait_stage = [&](int w) {
+                return mbar_wait(&bars->st_full[w % C::kStages],
+                                 (uint32_t)(w / C::kStages) & 1u, wd);
+            };
             bool ok = true;
-            if (n_items > 0) ok = mbar_wait(&bars->fixed_full, 0u, wd);
+            if (n_items > 0) {
+                ok = mbar_wait(&bars->fixed_full, 0u, wd) && wait_stage(0);
+                if (ok) {
+                    tc_fence_after();
+                    mma.rows_by_rows(C::kColS, dk0, st_k + q_off(0));               // S^T = K Q^T
+                    umma_commit(&bars->s_full);
+                    mma.rows_by_rows(C::kColDP, dv0, st_k + q_off(0) + kTileStep);  // dP^T = V dO^T
+                    umma_commit(&bars->dp_full);
+                }
+            }
             for (int w = 0; ok && w < n_items; ++w) {
-                const int slot = w % C::kStages;
-                ok = mbar_wait(&bars->st_full[slot], (uint32_t)(w / C::kStages) & 1u, wd);
+                ok = mbar_wait(&bars->p_done, (uint32_t)w & 1u, wd);
                 if (!ok) break;
                 tc_fence_after();
-                const uint64_t q_off = (uint64_t)slot * 2 * kTileStep;
-                mma.rows_by_rows(C::kColS, dk0, st_k + q_off);                // S^T  = K Q^T
-                mma.rows_by_rows(C::kColDP, dv0, st_k + q_off + kTileStep);   // dP^T = V dO^T
-                umma_commit(&bars->s_full);
-                ok = mbar_wait(&bars->p_full, (uint32_t)w & 1u, wd);
+                mma.tmem_by_tile(C::kColAcc0, C::kColS, st_mn + q_off(w) + kTileStep, w > 0);  // dV += P^T dO
+                if (w + 1 < n_items) {
+                    ok = wait_stage(w + 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    mma.rows_by_rows(C::kColS, dk0, st_k + q_off(w + 1));
+                    umma_commit(&bars->s_full);
+                }
+                ok = mbar_wait(&bars->ds_done, (uint32_t)w & 1u, wd);
                 if (!ok) break;
                 tc_fence_after();
-                mma.tmem_by_tile(C::kColAcc0, C::kColS, st_mn + q_off + kTileStep, w > 0);  // dV += P^T dO
-                mma.tmem_by_tile(C::kColAcc1, C::kColDP, st_mn + q_off, w > 0);             // dK += dS^T Q
-                umma_commit(&bars->st_empty[slot]);
+                mma.tmem_by_tile(C::kColAcc1, C::kColDP, st_mn + q_off(w), w > 0);             // dK += dS^T Q
+                umma_commit(&bars->st_empty[w % C::kStages]);
+                if (w + 1 < n_items) {
+                    mma.rows_by_rows(C::kColDP, dv0, st_k + q_off(w + 1) + kTileStep);
+                    umma_commit(&bars->dp_full);
+                }
             }
             umma_commit(&bars->acc_done);
             umma_commit(&bars->teardown);
@@ -363,7 +411,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int slot = w % C::kStages;
             const int g = w / nq;
             const int it = it0 + (w - g * nq);
-            // the stage's lse2 / D copies (their own barrier phase), then S and dP
+            // the stage's lse2 / D copies (their own barrier phase), then S
             ok = mbar_wait(&bars->st_full[slot], (uint32_t)(w / C::kStages) & 1u, wd);
             if (ok) ok = mbar_wait(&bars->s_full, (uint32_t)w & 1u, wd);
             ok = __all_sync(0xffffffffu, ok);
@@ -372,17 +420,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float* L2 = sCol + slot * 256;
             const float* DD = L2 + 128;
             const int q0 = it * 128;
-            bwd_softmax_half<true>(
-                tS, tDP, c0, c,
-                [&](int col) { return key_ok && (!p.causal || jr <= q0 + col); },
-                [&](int col, float (&l2)[4], float (&dd)[4]) {
+            float pv[64];
+            bwd_p_half<true>(
+                tS, c0, c, [&](int col) { return key_ok && (!p.causal || jr <= q0 + col); },
+                [&](int col, float (&l2)[4]) {
                     const float4 a = *reinterpret_cast<const float4*>(L2 + col);
-                    const float4 d = *reinterpret_cast<const float4*>(DD + col);
                     l2[0] = a.x; l2[1] = a.y; l2[2] = a.z; l2[3] = a.w;
-                    dd[0] = d.x; dd[1] = d.y; dd[2] = d.z; dd[3] = d.w;
-                });
+                },
+                pv);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            mbar_arrive(&bars->p_done);
+            ok = mbar_wait(&bars->dp_full, (uint32_t)w & 1u, wd);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            bwd_ds_half(tDP, c0, pv, [&](int col, float (&dd)[4]) {
+                const float4 d = *reinterpret_cast<const float4*>(DD + col);
+                dd[0] = d.x; dd[1] = d.y; dd[2] = d.z; dd[3] = d.w;
+            });
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_done);
         }
         if (ok) {
             ok = mbar_wait(&bars->acc_done, 0u, wd);
@@ -506,22 +565,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t st_k = smem_desc_sw128(smem_u32(sStage), 16, 1024);
             const uint64_t st_mn = smem_desc_sw128(smem_u32(sStage), C::kBlockBytes, 1024);
             constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
+            // Per item w: dP(w) | S read -> S(w+1) | dS(w) -> dQ(w), dP(w+1). S(w+1)
+            // is computed while the compute warps work on item w (they hold S(w)
+            // in registers once they signal p_done); dP(w+1) overwrites dS(w)
+            // after dQ(w) has read it (issue order).
+            auto k_off = [&](int w) { return (uint64_t)(w % C::kStages) * 2 * kTileStep; };
+            auto wait_stage = [&](int w) {
+                return mbar_wait(&bars->st_full[w % C::kStages],
+                                 (uint32_t)(w / C::kStages) & 1u, wd);
+            };
             bool ok = true;
-            if (n_items > 0) ok = mbar_wait(&bars->fixed_full, 0u, wd);
+            if (n_items > 0) {
+                ok = mbar_wait(&bars->fixed_full, 0u, wd) && wait_stage(0);
+                if (ok) {
+                    tc_fence_after();
+                    mma.rows_by_rows(C::kColS, dq0, st_k + k_off(0));                // S  = Q K^T
+                    umma_commit(&bars->s_full);
+                    mma.rows_by_rows(C::kColDP, ddo0, st_k + k_off(0) + kTileStep);  // dP = dO V^T
+                    umma_commit(&bars->dp_full);
+                }
+            }
             for (int w = 0; ok && w < n_items; ++w) {
-                const int slot = w % C::kStages;
-                ok = mbar_wait(&bars->st_full[slot], (uint32_t)(w / C::kStages) & 1u, wd);
+                if (w + 1 < n_items) {
+                    ok = mbar_wait(&bars->p_done, (uint32_t)w & 1u, wd) && wait_stage(w + 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    mma.rows_by_rows(C::kColS, dq0, st_k + k_off(w + 1));
+                    umma_commit(&bars->s_full);
+                }
+                ok = mbar_wait(&bars->ds_done, (uint32_t)w & 1u, wd);
                 if (!ok) break;
                 tc_fence_after();
-                const uint64_t k_off = (uint64_t)slot * 2 * kTileStep;
-                mma.rows_by_rows(C::kColS, dq0, st_k + k_off);                // S  = Q K^T
-                mma.rows_by_rows(C::kColDP, ddo0, st_k + k_off + kTileStep);  // dP = dO V^T
-                umma_commit(&bars->s_full);
-                ok = mbar_wait(&bars->p_full, (uint32_t)w & 1u, wd);
-                if (!ok) break;
-                tc_fence_after();
-                mma.tmem_by_tile(C::kColAcc0, C::kColDP, st_mn + k_off, w > 0);   // dQ += dS K
-                umma_commit(&bars->st_empty[slot]);
+                mma.tmem_by_tile(C::kColAcc0, C::kColDP, st_mn + k_off(w), w > 0);   // dQ += dS K
+                umma_commit(&bars->st_empty[w % C::kStages]);
+                if (w + 1 < n_items) {
+                    mma.rows_by_rows(C::kColDP, ddo0, st_k + k_off(w + 1) + kTileStep);
+                    umma_commit(&bars->dp_full);
+                }
             }
             umma_commit(&bars->acc_done);
             umma_commit(&bars->teardown);
@@ -546,18 +626,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const int k0 = w * 128;
-            bwd_softmax_half<false>(
-                tS, tDP, c0, c,
-                [&](int col) { return k0 + col < kv_lim && (!p.causal || k0 + col <= i); },
-                [&](int, float (&l2v)[4], float (&ddv)[4]) {
+            float pv[64];
+            bwd_p_half<false>(
+                tS, c0, c, [&](int col) { return k0 + col < kv_lim && (!p.causal || k0 + col <= i); },
+                [&](int, float (&l2v)[4]) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        l2v[e] = l2;
-                        ddv[e] = dd;
-                    }
-                });
+                    for (int e = 0; e < 4; ++e) l2v[e] = l2;
+                },
+                pv);
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            mbar_arrive(&bars->p_done);          // S(w) is in registers: S(w+1) may overwrite it
+            ok = mbar_wait(&bars->dp_full, (uint32_t)w & 1u, wd);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            bwd_ds_half(tDP, c0, pv, [&](int, float (&ddv)[4]) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ddv[e] = dd;
+            });
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_done);
         }
         if (ok) {
             ok = mbar_wait(&bars->acc_done, 0u, wd);
