@@ -214,9 +214,11 @@ __device__ __forceinline__ uint32_t bwd_setup(BwdBarriers* bars, const BwdParams
 // Phase 1: read S (fp32) and form P = exp2(s * c - lse2) on visible entries
 // (0 elsewhere) into pv; when kWriteP, also write P (bf16 pairs) to S's
 // columns [c0, c0 + 32). `visible(col)` tells whether column col of the row is
-// a visible (query, key) pair; `col_l2(col, l2)` gives lse2 of columns
+// a visible (query, key) pair, consulted only when kMask (tiles on the causal
+// diagonal or across kv_len; elsewhere every pair is visible and rows past N
+// get P = 0 from their lse2 = +inf); `col_l2(col, l2)` gives lse2 of columns
 // col..col+3 (pass A: per column; pass B: the row's own).
-template <bool kWriteP, typename Vis, typename ColL2>
+template <bool kWriteP, bool kMask, typename Vis, typename ColL2>
 __device__ __forceinline__ void bwd_p_half(uint32_t tS, int c0, float c, Vis visible,
                                            ColL2 col_l2, float (&pv)[64]) {
     uint32_t s0[32], s1[32];
@@ -231,7 +233,8 @@ __device__ __forceinline__ void bwd_p_half(uint32_t tS, int c0, float c, Vis vis
         for (int e = 0; e < 4; ++e) {
             const int qe = q + e;
             const float sv = __uint_as_float(qe < 32 ? s0[qe] : s1[qe - 32]);
-            pv[qe] = visible(c0 + qe) ? fast_exp2(fmaf(sv, c, -l2[e])) : 0.f;
+            const float pe = fast_exp2(fmaf(sv, c, -l2[e]));
+            pv[qe] = (!kMask || visible(c0 + qe)) ? pe : 0.f;
         }
     }
     if (kWriteP) {
@@ -405,6 +408,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t tDP = tmem + lane_base + C::kColDP;
         const int jr = jt * 128 + row;                 // this thread's key row
         const bool key_ok = jr < kv_lim;
+        const bool tile_masked = (jt + 1) * 128 > kv_lim;   // the key tile crosses kv_len
         const float c = p.scale_log2;
         bool ok = true;
         for (int w = 0; ok && w < n_items; ++w) {
@@ -421,13 +425,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float* DD = L2 + 128;
             const int q0 = it * 128;
             float pv[64];
-            bwd_p_half<true>(
-                tS, c0, c, [&](int col) { return key_ok && (!p.causal || jr <= q0 + col); },
-                [&](int col, float (&l2)[4]) {
-                    const float4 a = *reinterpret_cast<const float4*>(L2 + col);
-                    l2[0] = a.x; l2[1] = a.y; l2[2] = a.z; l2[3] = a.w;
-                },
-                pv);
+            auto vis = [&](int col) { return key_ok && (!p.causal || jr <= q0 + col); };
+            auto cl2 = [&](int col, float (&l2)[4]) {
+                const float4 a = *reinterpret_cast<const float4*>(L2 + col);
+                l2[0] = a.x; l2[1] = a.y; l2[2] = a.z; l2[3] = a.w;
+            };
+            if (tile_masked || (p.causal && it == jt))
+                bwd_p_half<true, true>(tS, c0, c, vis, cl2, pv);
+            else
+                bwd_p_half<true, false>(tS, c0, c, vis, cl2, pv);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_done);
@@ -627,13 +633,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             const int k0 = w * 128;
             float pv[64];
-            bwd_p_half<false>(
-                tS, c0, c, [&](int col) { return k0 + col < kv_lim && (!p.causal || k0 + col <= i); },
-                [&](int, float (&l2v)[4]) {
+            auto vis = [&](int col) { return k0 + col < kv_lim && (!p.causal || k0 + col <= i); };
+            auto cl2 = [&](int, float (&l2v)[4]) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) l2v[e] = l2;
-                },
-                pv);
+                for (int e = 0; e < 4; ++e) l2v[e] = l2;
+            };
+            if (k0 + 128 > kv_lim || (p.causal && w == it))
+                bwd_p_half<false, true>(tS, c0, c, vis, cl2, pv);
+            else
+                bwd_p_half<false, false>(tS, c0, c, vis, cl2, pv);
             tc_fence_before();
             mbar_arrive(&bars->p_done);          // S(w) is in registers: S(w+1) may overwrite it
             ok = mbar_wait(&bars->dp_full, (uint32_t)w & 1u, wd);
