@@ -22,7 +22,8 @@ rank 0 runs it.
 --backward times the backward pass (fa_bwd) on the workload's shape instead.
 --fp8 times the e4m3 forward (fa_fwd_fp8) on the workload's shape instead.
 --decode 1 times the split-KV path instead (one query row per head against an
-8K-key cache with grouped K/V heads), in GB/s of algorithmic bytes.
+8K-key cache with grouped K/V heads), in GB/s of algorithmic bytes; --decode 2 the
+same for one sequence against a 128K-key cache (keys split into ranges and merged).
 """
 from __future__ import annotations
 

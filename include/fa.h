@@ -133,12 +133,12 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *
 size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits);
 
 /*
- * A num_splits for fa_fwd_splitkv on the current device. Work units (one per
- * head group, row block and range) are equal-sized, so this is the fewest
- * ranges, each at least four 128-key tiles long and at most FA_MAX_SPLITS,
- * that make at least one full wave of units over the SMs with the last wave at
- * least 90 % full (else the best-filled count). Returns 1 for invalid
- * arguments. Reads only device attributes.
+ * A num_splits for fa_fwd_splitkv on the current device: the fewest key
+ * ranges that give at least 85 % of one wave of work units (one per head group,
+ * row block and range) over the SMs, each range at least four 128-key tiles
+ * long and at most FA_MAX_SPLITS (every unit pays a fixed cost, so fewer,
+ * longer units win once most SMs are busy). Returns 1 for invalid arguments.
+ * Reads only device attributes.
  */
 int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
 

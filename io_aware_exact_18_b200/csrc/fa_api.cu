@@ -497,23 +497,14 @@ FA_EXPORT int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, 
     const int64_t n_rb = ((int64_t)Nq + nq_blk - 1) / nq_blk;
     const int64_t base = (int64_t)B * (H / G) * n_rb;
     const int64_t key_tiles = ((int64_t)Nk + fa::kTile - 1) / fa::kTile;
-    // Units are equal-sized, so the last wave decides: take the fewest ranges
-    // (each at least four key tiles) that give at least one full wave of
-    // units with the last wave >= 90 % busy; else the best-filled count.
+    // Each unit pays a fixed cost (its Q tile, the first scores, the epilogue and
+    // the partials the merge reads back), so use as few ranges as keep most of
+    // the SMs busy: the fewest that give at least 85 % of one wave of units,
+    // each range at least four key tiles long.
     const int64_t s_max = std::min<int64_t>(fa::kMaxSplits, std::max<int64_t>(1, key_tiles / 4));
-    int64_t best = 1;
-    double best_eff = -1.0;
-    for (int64_t sp = 1; sp <= s_max; ++sp) {
-        const int64_t units = base * sp;
-        const int64_t waves = (units + sms - 1) / sms;
-        const double eff = (double)units / (double)(waves * sms);
-        if (units >= sms && eff >= 0.9) return (int)sp;
-        if (eff > best_eff + 1e-9) {
-            best_eff = eff;
-            best = sp;
-        }
-    }
-    return (int)best;
+    const int64_t want = (int64_t)(0.85 * sms + 0.999);
+    const int64_t sp = (want + base - 1) / base;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(sp, s_max));
 }
 
 FA_EXPORT int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,

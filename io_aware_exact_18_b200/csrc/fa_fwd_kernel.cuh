@@ -108,7 +108,7 @@ struct Cfg {
     static constexpr int kSlots =                         // K/V ring depth
         (E == 1) ? 8 : (D == 256) ? 2 : (D == 128) ? (QT == 2 ? 4 : 5) : 8;
     static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
-    static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 1024 /*barriers*/;
+    static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 3072 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr int kUnitConsumers = 1 + 4 * kQT;   // MMA thread + one lane per softmax warp
     // S buffer b (a query tile's, or with one tile the buffer of key-tile parity b)
@@ -155,13 +155,16 @@ struct SmemBarriers {
     uint64_t teardown;
     uint64_t kv_full[8];
     uint64_t kv_empty[8];
+    uint64_t merge_full[2];    // two-accumulator mode: warpgroup 1's (m, l) per row, by unit parity
+    float merge_m[2][kTile];
+    float merge_l[2][kTile];
     uint4 clc_resp[2];         // 16-byte aligned (offset is a multiple of 16)
     int unit_id[2];
     uint32_t tmem_base;
     int abort;
     int skip;
 };
-static_assert(sizeof(SmemBarriers) <= 1024, "barrier region");
+static_assert(sizeof(SmemBarriers) <= 3072, "barrier region");
 static_assert(offsetof(SmemBarriers, clc_resp) % 16 == 0, "CLC response alignment");
 
 // One work unit, decoded from its launch-order index. A tile's 128 rows hold
@@ -300,6 +303,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = Cfg<D, QT, E>;
     const Shape<kGen> sh(p);
+    // Two-accumulator mode (the general kernel at d <= 128): the one query tile's
+    // key tiles alternate between the two softmax warpgroups, each with its own
+    // reference maximum, running sum and O accumulator (TMEM: Sa | Sb | O0 | O1);
+    // the epilogue merges the two halves by their log-sum-exp, as the split-KV
+    // merge does. It keeps both warpgroups busy when a unit has one live tile.
+    constexpr bool kDual = kGen && QT == 1 && D <= 128;
+    constexpr int kSoftmaxWarps = 4 * (kDual ? 2 : QT);
+    constexpr int kConsumers = 1 + kSoftmaxWarps;   // MMA thread + one lane per softmax warp
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -322,7 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->o_done[t], 1);
             mbar_init(&bars->o_empty[t], kTile);
             mbar_init(&bars->unit_full[t], 1);
-            mbar_init(&bars->unit_empty[t], C::kUnitConsumers);
+            mbar_init(&bars->unit_empty[t], kConsumers);
+            mbar_init(&bars->merge_full[t], kTile);
             mbar_init(&bars->clc_bar[t], 1);
         }
         mbar_init(&bars->teardown, 1);
@@ -593,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (id < 0) break;
                 const Unit u = decode_unit<C::kQT, kGen>(id, p);
                 const int n = u.n[0];
-                bool o_ready = (k == 0);
+                bool o_ready[2] = {k == 0, k == 0};
                 // positions of K_t and V_j in this unit's load order (see the producer)
                 auto posK = [&](int t) { return t < 2 ? t : 2 * t - 1; };
                 auto posV = [&](int j) { return (j <= n - 3) ? 2 + 2 * j : n + j; };
@@ -619,14 +631,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     ok = mbar_wait(&bars->p_full[b], ph_p[b] & 1u, wd);
                     ++ph_p[b];
-                    if (ok && !o_ready) {
-                        ok = mbar_wait(&bars->o_empty[0], (uint32_t)((k - 1) & 1), wd);
-                        o_ready = true;
+                    const int ob = kDual ? b : 0;          // O accumulator of this tile
+                    if (ok && !o_ready[ob]) {
+                        ok = mbar_wait(&bars->o_empty[ob], (uint32_t)((k - 1) & 1), wd);
+                        o_ready[ob] = true;
                     }
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(0, b, slot_of(posV(j)), j > 0);
-                    umma_commit(&bars->o_done[0]);
+                    issue_pv(ob, b, slot_of(posV(j)), kDual ? j > 1 : j > 0);
+                    umma_commit(&bars->o_done[ob]);
                     umma_commit(&bars->kv_empty[slot_of(posV(j))]);
                     if (j + 2 < n) {
                         ok = wait_load(posK(j + 2));
@@ -639,10 +652,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (!ok) break;
-                if (n == 0) {                          // idle unit: its once-per-unit hand-offs
-                    umma_commit(&bars->q_empty[0]);
-                    if (!o_ready) ok = mbar_wait(&bars->o_empty[0], (uint32_t)((k - 1) & 1), wd);
-                    umma_commit(&bars->o_done[0]);
+                if (n == 0) umma_commit(&bars->q_empty[0]);   // idle unit: its Q hand-off
+                // an O accumulator that took no tile this unit: its once-per-unit hand-offs
+                for (int ob = 0; ok && ob < (kDual ? 2 : 1); ++ob) {
+                    if (n > ob) continue;
+                    if (!o_ready[ob])
+                        ok = mbar_wait(&bars->o_empty[ob], (uint32_t)((k - 1) & 1), wd);
+                    umma_commit(&bars->o_done[ob]);
                 }
                 L0 += 2 * n;
             }
@@ -652,12 +668,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_drain(&bars->teardown, 0u, wd);
         }
         __syncwarp();
-    } else if (warp < 4 * C::kQT) {
+    } else if (warp < kSoftmaxWarps) {
         // ====================================================== softmax warpgroups
-        const int t = warp >> 2;                      // query tile 0 or 1
+        const int wg = warp >> 2;                     // warpgroup
+        const int t = kDual ? 0 : wg;                 // query tile 0 or 1
+        const int ob = wg;                            // O accumulator / o_done of this warpgroup
         const int row = tid & (kTile - 1);            // row within the tile == TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tO = tmem + lane_base + C::col_o(t);
+        const uint32_t tO = tmem + lane_base + C::col_o(ob);
         const float c = p.scale_log2;
         uint32_t ph_s[2] = {0u, 0u};   // s_full phases consumed (per S buffer)
         uint32_t o_base = 0;   // o_done phases of earlier units
@@ -690,8 +708,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool idle_warp = kGen && !__any_sync(0xffffffffu, row_id >= 0);
             float m_ref = -INFINITY;   // reference maximum (raw score units)
             float l = 0.f;             // running sum of exp2((s - m_ref) * c)
+            // tiles of this warpgroup: all of them, or (two accumulators) j = wg, wg + 2, ...
+            const int j_first = kDual ? wg : 0, j_step = kDual ? 2 : 1;
+            const int n_own = kDual ? (n > wg ? (n - wg + 1) / 2 : 0) : n;
 
-            for (int j = 0; j < n; ++j) {
+            for (int j = j_first; j < n; j += j_step) {
+                const int jo = kDual ? (j - wg) / 2 : j;       // index among this warpgroup's tiles
                 const int sb = (C::kQT == 2) ? t : (j & 1);   // this tile's S buffer
                 const uint32_t tS = tmem + lane_base + C::col_s(sb);
                 ok = mbar_wait(&bars->s_full[sb], ph_s[sb] & 1u, wd);
@@ -747,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (__any_sync(0xffffffffu, rescale)) {
                     // O holds the P.V sums of tiles < j: wait for the last of them,
                     // then bring it to the new reference maximum.
-                    ok = mbar_wait(&bars->o_done[t], (o_base + (uint32_t)(j - 1)) & 1u, wd);
+                    ok = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(jo - 1)) & 1u, wd);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     tc_fence_after();
@@ -769,10 +791,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
 
             // ------------------------------------------------ epilogue
-            // the unit's last o_done phase for this tile (its idle phase if n == 0)
-            const uint32_t last = o_base + (uint32_t)(n > 0 ? n - 1 : 0);
-            o_base += (uint32_t)(n > 0 ? n : 1);
-            if (C::kQT == 1 && n >= 2) {
+            // the unit's last o_done phase for this accumulator (its idle phase if none)
+            const uint32_t last = o_base + (uint32_t)(n_own > 0 ? n_own - 1 : 0);
+            o_base += (uint32_t)(n_own > 0 ? n_own : 1);
+            if (!kDual && C::kQT == 1 && n >= 2) {
                 // With one query tile the last score tile was issued after
                 // P.V(n-3) only, so o_done may still be in phase n-2: a parity
                 // wait for phase n-1 alone would pass at once. Wait in order.
@@ -780,9 +802,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
             }
-            ok = mbar_wait(&bars->o_done[t], last & 1u, wd);
+            ok = mbar_wait(&bars->o_done[ob], last & 1u, wd);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
+            // Two accumulators: warpgroup 1 hands its row's (m, l) to warpgroup 0
+            // (its O1 is complete: it has just waited for its last P.V), and
+            // warpgroup 0 writes the merged row.
+            float a0 = 1.f, a1 = 0.f;          // weights of O0 and O1 in the merged row
+            bool have1 = false;                // O1 holds a tile of this unit
+            if constexpr (kDual) {
+                const int mb = k & 1;
+                if (wg == 1) {
+                    bars->merge_m[mb][row] = (l > 0.f) ? m_ref * c : -INFINITY;
+                    bars->merge_l[mb][row] = l;
+                    mbar_arrive(&bars->merge_full[mb]);
+                    continue;
+                }
+                ok = mbar_wait(&bars->merge_full[mb], (uint32_t)((k >> 1) & 1), wd);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                const float m0 = (l > 0.f) ? m_ref * c : -INFINITY;
+                const float m1 = bars->merge_m[mb][row], l1 = bars->merge_l[mb][row];
+                const float mm = fmaxf(m0, m1);
+                a0 = (l > 0.f) ? fast_exp2(m0 - mm) : 0.f;
+                a1 = (l1 > 0.f) ? fast_exp2(m1 - mm) : 0.f;
+                l = l * a0 + l1 * a1;
+                m_ref = (mm == -INFINITY) ? -INFINITY : mm / c;   // merged reference (score units)
+                have1 = n > 1;
+            }
             tc_fence_after();
             const bool write = row_id >= 0;
             const float inv_l = (l > 0.f) ? p.o_mul / l : 0.f;
@@ -794,7 +841,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t r[32];
                 if (n > 0 && !idle_warp) {
                     tmem_ld32(tO + (uint32_t)(ch * 32), r);
-                    tmem_wait_ld();
+                    if constexpr (kDual) {
+                        uint32_t r1[32];
+                        if (have1) {
+                            tmem_ld32(tmem + lane_base + C::col_o(1) + (uint32_t)(ch * 32), r1);
+                            tmem_wait_ld();
+                        } else {
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) r1[q] = 0u;
+                        }
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            r[q] = __float_as_uint(__uint_as_float(r[q]) * a0 +
+                                                   __uint_as_float(r1[q]) * a1);
+                    } else {
+                        tmem_wait_ld();
+                    }
                 } else {
 #pragma unroll
                     for (int q = 0; q < 32; ++q) r[q] = 0u;
@@ -802,7 +865,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ch == D / 32 - 1) {
                     // O has been read: the next unit's first P.V may overwrite it
                     tc_fence_before();
-                    mbar_arrive(&bars->o_empty[t]);
+                    mbar_arrive(&bars->o_empty[ob]);
+                    if (kDual) mbar_arrive(&bars->o_empty[1]);
                 }
                 if (write && (!kGen || p.o_part == nullptr)) {
                     uint4* dst = reinterpret_cast<uint4*>(p.o + orow_idx * D + ch * 32);

@@ -115,12 +115,28 @@ def test_square_single_range_matches_fa_fwd_bitwise(fa):
 
 def test_decode_workload_full_size(fa):
     """The decode workload the benchmark times, every row checked, at the
-    split count the benchmark uses (the library's default)."""
+    split count the benchmark uses (the library's default) and at 8 ranges."""
     w = workloads.DECODE_WORKLOADS[0]
+    q, k, v, _ = workloads.make_qkv(w.B, w.H, w.H_kv, w.Nq, w.Nk, w.d, seed=w.seed)
+    splits = fa.fa_splitkv_default_splits(w.B, w.H, w.H_kv, w.Nq, w.Nk, w.d)
+    for sp in sorted({splits, 8}):
+        check(fa, q, k, v, w.causal, sp, what=f"{w.name} splits={sp}")
+
+
+def test_long_cache_decode_workload_sampled(fa):
+    """The 128K-key decode workload at the default (split) range count, all
+    32 heads' single rows checked against the oracle."""
+    w = workloads.DECODE_WORKLOADS[1]
     q, k, v, _ = workloads.make_qkv(w.B, w.H, w.H_kv, w.Nq, w.Nk, w.d, seed=w.seed)
     splits = fa.fa_splitkv_default_splits(w.B, w.H, w.H_kv, w.Nq, w.Nk, w.d)
     assert splits > 1
     check(fa, q, k, v, w.causal, splits, what=f"{w.name} splits={splits}")
+
+
+def test_default_splits_fill_the_device(fa):
+    """One long-context head group needs many ranges; a large batch needs one."""
+    assert fa.fa_splitkv_default_splits(1, 32, 8, 1, 131072, 128) >= 8
+    assert fa.fa_splitkv_default_splits(64, 32, 8, 1, 8192, 128) == 1
 
 
 def test_splits_are_deterministic(fa):

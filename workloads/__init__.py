@@ -161,6 +161,10 @@ class DecodeWorkload:
 # specialised kernels target ("FlashAttention (UR)", "Specialised solutions").
 DECODE_WORKLOADS = [
     DecodeWorkload("decode_gqa_B16_H32_Hkv8_Nq1_Nk8192_d128", 16, 32, 8, 1, 8192, 128),
+    # one sequence against a 128K-token cache: too few head groups to fill the
+    # SMs, so the keys are split into ranges and merged
+    DecodeWorkload("decode_gqa_B1_H32_Hkv8_Nq1_Nk131072_d128", 1, 32, 8, 1, 131072, 128,
+                   seed=12),
 ]
 DECODE_BY_NAME = {w.name: w for w in DECODE_WORKLOADS}
 
