@@ -377,6 +377,17 @@ def our_arm(args, w):
         raise fa.FAError(st, "e2e")
     e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
 
+    # ---- visible (query, key) pairs: the exponentials the method needs and the
+    # FLOPs of the keys that are not masked (the metric counts nominal FLOPs)
+    import numpy as np
+    vis = 0
+    kv_lims = [w.N] * w.B if kv_len is None else [min(max(int(x), 0), w.N) for x in kv_len]
+    rows = np.arange(w.N, dtype=np.int64)
+    for lim in kv_lims:
+        vis += int(np.minimum(lim, rows + 1).sum()) if w.causal else lim * w.N
+    vis *= w.H
+    eff_flops = 4.0 * w.d * vis
+
     # ---- roofline of the (only) kernel: one launch per step
     peaks, peak_src = load_peaks()
     achieved = flops / (ms_local * 1e-3) / 1e12
@@ -389,6 +400,14 @@ def our_arm(args, w):
                 "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
                 "algorithmic_bytes": float(w.B * w.N * (2 * w.H * w.d * 2 + 2 * w.kv_heads * w.d * 2
                                                         + 4 * w.H)),
+                "traffic_over_algorithmic": (None if traffic is None else traffic / float(
+                    w.B * w.N * (2 * w.H * w.d * 2 + 2 * w.kv_heads * w.d * 2 + 4 * w.H))),
+                # secondary bound: one exponential per visible score; MUFU ex2 runs 16 per
+                # clock per SM (148 SMs) at the sampled SM clock
+                "exp_per_s": vis / (ms_local * 1e-3),
+                "exp_frac_of_mufu": vis / (ms_local * 1e-3) / (
+                    16 * 148 * float(clocks.get("sm_mhz") or 1965) * 1e6),
+                "effective_tflops_visible_keys": eff_flops / (ms_local * 1e-3) / 1e12,
                 "kernel": f"fa_fwd_sm100<{w.d},{1 if w.d == 256 else 2},square>"}
 
     cpu = None
