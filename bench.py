@@ -63,10 +63,16 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """sha256/16 of the forward kernel's sources with comments and blank space
+    removed, so that edits to comments alone keep a recorded measurement."""
+    import re
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

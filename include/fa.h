@@ -1,5 +1,6 @@
 /*
- * fa.h -- C ABI of the exact, fused attention forward library (libfa.so).
+ * fa.h -- C ABI of the exact, fused attention library (libfa.so): the forward
+ * (square, grouped heads, split-KV decoding, e4m3 inputs) and its backward.
  *
  * The operation is the attention of "FlashAttention (UR)", section "Problem
  * of standard attention":

@@ -1,6 +1,6 @@
 // Host side of libfa.so: argument validation, TMA descriptor encoding and the
-// launch of the fused forward kernel. Declarations and the contract are in
-// include/fa.h.
+// launches of the forward (square, split-KV with its merge, e4m3), backward
+// and diagnostic kernels. Declarations and the contract are in include/fa.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

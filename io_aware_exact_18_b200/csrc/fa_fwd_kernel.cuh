@@ -1,7 +1,8 @@
 // Fused exact attention forward for sm_100a (B200).
 //
 // Computes O = softmax(scale * Q K^T + mask) V and lse = ln sum_j exp(s_ij)
-// for bf16 Q, K, V laid out [B, H, N, d] (d innermost), accumulating in fp32.
+// for bf16 (or e4m3, with per-tensor descales) Q, K, V laid out [B, H, N, d]
+// (d innermost), accumulating in fp32.
 // The N x N score matrix never leaves the SM: each 128 x 128 score tile lives
 // in tensor memory (TMEM), is turned into probabilities there, and feeds the
 // P.V product directly ("FlashAttention (UR)", sections "Tiling and block
@@ -44,23 +45,32 @@
 // from its query head's group head, and neighbouring query heads (same group)
 // run next to each other so the shared K/V stays in L2.
 //
+// Instantiations fa_fwd_sm100<D, QT, kGen, E>: head dim D; QT query tiles per
+// unit (2 at d <= 128 for square attention; 1 with S double-buffered at
+// d = 256 and in the general kernel); kGen the general (split-KV) form; E the
+// element bytes of Q, K, V (2: bf16, 1: e4m3 with kind::f8f6f4 products).
+//
 // Roles inside a CTA (320 threads):
 //   warps 0-3   softmax for query tile 0 (thread r owns row r = TMEM lane r)
-//   warps 4-7   softmax for query tile 1
+//   warps 4-7   softmax for query tile 1 (QT = 2), or for the odd key tiles of
+//               the one query tile (general kernel at d <= 128), or idle
 //   warp  8     issues tcgen05 MMAs (one thread) and owns the TMEM allocation
 //   warp  9     issues TMA loads and the unit requests (one thread)
 // With one thread per row no cross-thread reduction is needed for the row
 // max and row sum. The two softmax warpgroups ping-pong: while one works on
 // its score tile the tensor cores run the other tile's P.V and next Q.K^T.
 //
-// TMEM (512 columns x 128 lanes of 32 bit):
+// TMEM (512 columns x 128 lanes of 32 bit), QT = 2:
 //   [0,128)    S0 (fp32 scores of tile 0); P0 (bf16 pairs) overwrites [0,64)
 //   [128,256)  S1 / P1
 //   [256,256+d)      O0 accumulator (fp32)
 //   [256+d,256+2d)   O1 accumulator
-// Shared memory: Q0, Q1 and a ring of K/V slots, each a 128-row tile stored
-// as d/64 column blocks of 128 rows x 128 bytes in the 128-byte swizzled
-// layout that TMA writes and tcgen05 descriptors read.
+// QT = 1: Sa | Sb (alternate key tiles) | O, or | O0 | O1 in the general kernel
+// at d <= 128, where each softmax warpgroup keeps its own accumulator and the
+// epilogue merges the two by log-sum-exp. e4m3 P takes 32 columns.
+// Shared memory: the Q tiles and a ring of K/V slots, each a 128-row tile
+// stored as 128-byte column blocks of 128 rows in the 128-byte swizzled layout
+// that TMA writes and tcgen05 descriptors read; then the barriers.
 //
 // Synchronisation (mbarriers; every wait is bounded). Each barrier's phases
 // are counted per role across units; per unit and tile there is exactly one
@@ -110,7 +120,6 @@ struct Cfg {
     static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 3072 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr int kUnitConsumers = 1 + 4 * kQT;   // MMA thread + one lane per softmax warp
     // S buffer b (a query tile's, or with one tile the buffer of key-tile parity b)
     __device__ static constexpr uint32_t col_s(int b) { return (uint32_t)(b * 128); }
     __device__ static constexpr uint32_t col_o(int t) { return 256u + (uint32_t)(t * D); }
