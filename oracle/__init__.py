@@ -66,6 +66,10 @@ def _bind(lib):
     lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, u16p, u16p, u16p, u16p, dp, dp, dp, c_int,
                                     c_int, c_int, c_int, c_int, c_double, c_int, i32p, c_int]
     lib.oracle_attn_bwd.restype = c_int
+    lib.oracle_attn_bwd_dq_rows.argtypes = [u16p, u16p, u16p, u16p, dp, c_int, c_int, c_int,
+                                            c_int, c_int, c_double, c_int, i32p, i32p, c_int,
+                                            c_int]
+    lib.oracle_attn_bwd_dq_rows.restype = c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     return lib
@@ -203,3 +207,35 @@ def attention_bwd(q, k, v, do, scale, causal=False, kv_len=None, nthreads=0, lib
     if rc != 0:
         raise RuntimeError(f"oracle returned error {rc}")
     return dq, dk, dv
+
+
+def attention_bwd_dq_rows(q, k, v, do, scale, rows, causal=False, kv_len=None, nthreads=0,
+                          lib=None):
+    """dQ of the given query rows of every (b, h), in fp64: [B, H, len(rows), d].
+    Same definition as attention_bwd (dQ row i needs row i's P, dP and D only);
+    bf16 torch tensors or uint16 arrays."""
+    lib = lib or load()
+    arrs = [_as_numpy(x) for x in (q, k, v, do)]
+    if not all(b for _, b in arrs):
+        raise TypeError("q, k, v, do must be bf16")
+    (qa, _), (ka, _), (va, _), (da, _) = arrs
+    B, H, N, d = qa.shape
+    Hkv = ka.shape[1]
+    if ka.shape != (B, Hkv, N, d) or va.shape != ka.shape or da.shape != qa.shape:
+        raise ValueError("bad shapes")
+    ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    kvp = None
+    if kv_len is not None:
+        kvl = np.ascontiguousarray(np.asarray(
+            kv_len.cpu().numpy() if hasattr(kv_len, "cpu") else kv_len, dtype=np.int32))
+        kvp = kvl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    out = np.zeros((B, H, len(ra), d), dtype=np.float64)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    rc = lib.oracle_attn_bwd_dq_rows(*(a.ctypes.data_as(u16p) for a in (qa, ka, va, da)),
+                                     out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), B, H,
+                                     Hkv, N, d, float(scale), int(bool(causal)), kvp,
+                                     ra.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                     len(ra), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle returned error {rc}")
+    return out

@@ -391,6 +391,78 @@ int oracle_attn_bwd(const double *qd, const double *kd, const double *vd, const 
     return err;
 }
 
+/*
+ * dQ of selected query rows only (same definition as oracle_attn_bwd, which
+ * dQ row i depends on through row i alone: its P, dP and D). For checks at
+ * sizes where the full backward is out of reach. dq_rows: [B,H,nrows,d].
+ * bf16 inputs only.
+ */
+int oracle_attn_bwd_dq_rows(const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
+                            const uint16_t *dob, double *dq_rows, int B, int H, int Hkv, int N,
+                            int d, double scale, int causal, const int32_t *kv_len,
+                            const int32_t *rows, int nrows, int nthreads)
+{
+    if (!qb || !kb || !vb || !dob || !dq_rows || !rows) return ORACLE_EINVAL;
+    int rc = check_args(B, H, N, d, scale, causal);
+    if (rc) return rc;
+    if (B == 0 || H == 0 || N == 0 || nrows == 0) return ORACLE_OK;
+    if (Hkv <= 0 || Hkv > H || H % Hkv != 0 || nrows < 0) return ORACLE_EINVAL;
+    for (int r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= N) return ORACLE_EINVAL;
+    const size_t head = (size_t)N * d;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        /* per thread: one K/V head, and scratch for the dK/dV sums it discards */
+        double *buf = (double *)malloc((4 * head + 4 * (size_t)d + 2 * (size_t)N) * sizeof(double));
+        if (!buf) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        } else {
+            double *K = buf, *V = buf + head, *dKs = buf + 2 * head, *dVs = buf + 3 * head;
+            double *qi = buf + 4 * head, *doi = qi + d;
+            double *prow = doi + 2 * (size_t)d, *dsrow = prow + N;
+            int loaded = -1;
+#pragma omp for schedule(dynamic, 1)
+            for (int bh = 0; bh < B * H; ++bh) {
+                const int b = bh / H, h = bh % H;
+                const int g = b * Hkv + h / (H / Hkv);
+                int kv_lim = N;
+                if (kv_len) {
+                    kv_lim = kv_len[b];
+                    if (kv_lim < 0) kv_lim = 0;
+                    if (kv_lim > N) kv_lim = N;
+                }
+                if (g != loaded) {
+                    for (size_t e = 0; e < head; ++e) {
+                        K[e] = bf16_to_f64(kb[(size_t)g * head + e]);
+                        V[e] = bf16_to_f64(vb[(size_t)g * head + e]);
+                    }
+                    loaded = g;
+                }
+                for (int r = 0; r < nrows; ++r) {
+                    const int i = rows[r];
+                    const size_t qoff = ((size_t)bh * N + i) * d;
+                    for (int t = 0; t < d; ++t) {
+                        qi[t] = bf16_to_f64(qb[qoff + t]);
+                        doi[t] = bf16_to_f64(dob[qoff + t]);
+                    }
+                    for (size_t e = 0; e < head; ++e) dKs[e] = dVs[e] = 0.0;
+                    bwd_one_row(qi, doi, K, V, N, d, scale, i, causal, kv_lim, prow, dsrow,
+                                dq_rows + ((size_t)bh * nrows + r) * d, dKs, dVs);
+                }
+            }
+            free(buf);
+        }
+    }
+    return err;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -125,8 +125,22 @@ def pin_bwd_bf16_inputs_equal_f64(lib):
         assert np.array_equal(x, y)
 
 
+def pin_bwd_dq_rows_equal_full(lib):
+    """The row-subset driver gives exactly the full backward's dQ rows."""
+    import torch
+    g = torch.Generator().manual_seed(16)
+    q, do = (torch.randn(2, 4, 33, 8, generator=g).to(torch.bfloat16) for _ in range(2))
+    k, v = (torch.randn(2, 2, 33, 8, generator=g).to(torch.bfloat16) for _ in range(2))
+    rows = [0, 5, 17, 32]
+    for causal, kv_len in ((True, None), (False, [20, 33])):
+        full, _, _ = _bwd(lib, q, k, v, do, 0.4, causal, kv_len)
+        part = oracle.attention_bwd_dq_rows(q, k, v, do, 0.4, rows, causal=causal,
+                                            kv_len=kv_len, nthreads=1, lib=lib)
+        assert np.array_equal(part, full[:, :, rows]), (causal, kv_len)
+
+
 PINS = [pin_bwd_finite_differences, pin_bwd_torch_autograd, pin_bwd_invariants,
-        pin_bwd_zero_output_gradient, pin_bwd_bf16_inputs_equal_f64]
+        pin_bwd_zero_output_gradient, pin_bwd_bf16_inputs_equal_f64, pin_bwd_dq_rows_equal_full]
 
 
 def failures(lib):
