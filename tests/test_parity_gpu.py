@@ -168,13 +168,21 @@ def test_head_dim_256_sampled_full_size(fa):
 def test_grouped_and_multi_query(fa, H, H_kv, d, causal):
     """K/V heads shared by groups of query heads (H_kv = 1: multi-query)."""
     B, N = 3, 333
-    g = torch.Generator().manual_seed(1000 + H * 10 + H_kv + d + causal)
-    q = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
-    k = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
-    v = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+    q, k, v, _ = workloads.make_qkv(B, H, H_kv, N, N, d, seed=1000 + H * 10 + H_kv + d + causal)
     kv_len = torch.tensor([333, 200, 0], dtype=torch.int32)
     check_full(fa, q, k, v, causal, kv_len, what=f"H={H} H_kv={H_kv} d={d} causal={causal}")
     check_full(fa, q, k, v, causal, None, what=f"H={H} H_kv={H_kv} d={d} causal={causal}")
+
+
+def test_grouped_heads_sampled_full_size(fa):
+    """The grouped-heads long-context launch the benchmark measures (B1 H32
+    H_kv8 N16384 d128 causal): sampled rows of every head against the oracle."""
+    B, H, H_kv, N, d = 1, 32, 8, 16384, 128
+    q, k, v, _ = workloads.make_qkv(B, H, H_kv, N, N, d, seed=3208)
+    o, lse = run_gpu(fa, q, k, v, True)
+    rows = workloads.sample_rows(N, seed=8, n_random=32, edge=16)
+    o_ref, lse_ref = oracle.attention(q, k, v, 1 / math.sqrt(d), causal=True, rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], o_ref, lse_ref, "H32 H_kv8 N16384 causal")
 
 
 def test_peaky_rows_rescale(fa):
