@@ -266,3 +266,14 @@ def test_invalid_arguments_on_device(fa):
         fa.attention(x, x, x)
     assert e.value.status == fa.FA_ERR_UNSUPPORTED
     assert fa.fa_last_device_error(None) == fa.FA_OK
+
+
+def test_very_long_sequence_sampled(fa):
+    """N = 131072 (1024 query tiles per head, units far past the SM count):
+    sampled rows of every head against the oracle."""
+    B, H, N, d = 1, 4, 131072, 128
+    q, k, v, _ = workloads.make_custom(B, H, N, d, seed=131)
+    o, lse = run_gpu(fa, q, k, v, True)
+    rows = workloads.sample_rows(N, seed=13, n_random=24, edge=4)
+    o_ref, lse_ref = oracle.attention(q, k, v, 1 / math.sqrt(d), causal=True, rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], o_ref, lse_ref, "N=131072 causal")

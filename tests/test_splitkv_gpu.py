@@ -161,3 +161,13 @@ def test_splitkv_guard_regions_untouched(fa):
     torch.cuda.synchronize()
     for buf, n in ((o_buf, n_o), (l_buf, n_l)):
         assert torch.all(buf[:pad] == 7.0) and torch.all(buf[pad + n:] == 7.0)
+
+
+def test_decode_million_key_cache(fa):
+    """One query row per head against 2^20 keys (8192 key tiles), at the
+    library's default range count: every row against the oracle."""
+    B, H, H_kv, Nq, Nk, d = 1, 16, 4, 1, 1 << 20, 128
+    q, k, v, _ = workloads.make_qkv(B, H, H_kv, Nq, Nk, d, seed=20)
+    splits = fa.fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d)
+    assert splits > 1
+    check(fa, q, k, v, True, splits, what=f"Nk=2^20 splits={splits}")
