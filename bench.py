@@ -96,6 +96,19 @@ def recorded_traffic(workload_name: str):
         return None
 
 
+def visible_pairs(w, kv_len=None) -> int:
+    """Number of visible (query row, key) pairs over all B*H heads of a square
+    workload: key j is visible to row i iff j < kv_len[b] (clamped to [0, N])
+    and, when causal, j <= i."""
+    import numpy as np
+    kv_lims = [w.N] * w.B if kv_len is None else [min(max(int(x), 0), w.N) for x in kv_len]
+    rows = np.arange(w.N, dtype=np.int64)
+    vis = 0
+    for lim in kv_lims:
+        vis += int(np.minimum(lim, rows + 1).sum()) if w.causal else lim * w.N
+    return vis * w.H
+
+
 class ClockSampler:
     """Samples SM clock, power and clock-event (throttle) reasons in a
     background thread through NVML every 20 ms; read-only queries."""
@@ -385,13 +398,7 @@ def our_arm(args, w):
 
     # ---- visible (query, key) pairs: the exponentials the method needs and the
     # FLOPs of the keys that are not masked (the metric counts nominal FLOPs)
-    import numpy as np
-    vis = 0
-    kv_lims = [w.N] * w.B if kv_len is None else [min(max(int(x), 0), w.N) for x in kv_len]
-    rows = np.arange(w.N, dtype=np.int64)
-    for lim in kv_lims:
-        vis += int(np.minimum(lim, rows + 1).sum()) if w.causal else lim * w.N
-    vis *= w.H
+    vis = visible_pairs(w, kv_len)
     eff_flops = 4.0 * w.d * vis
 
     # ---- roofline of the (only) kernel: one launch per step
