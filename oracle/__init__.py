@@ -11,6 +11,10 @@ Two independent routes to the same result:
 * :func:`attention_bwd` -- the gradients dQ, dK, dV of the same definition for
   a given dO (chain rule through the row softmax, one query row at a time), in
   fp64 C. The pages state no backward algorithm; this is the exact gradient.
+* :func:`attention_bwd_dq_rows` -- dQ of selected query rows only (the same
+  definition; dQ row i depends on row i alone), for checks at full size.
+* :mod:`oracle.fp8` -- e4m3 decoding by the format's definition, feeding the
+  fp64 attention of the dequantized tensors.
 * :func:`online.attention_online` -- a blockwise online-softmax evaluation in
   numpy (running row max and running sum of exponentials, rescaled per key
   block), following section "Online softmax" of the same page. It exists only

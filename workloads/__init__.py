@@ -20,6 +20,13 @@ Recipe (fixed, so any run can be reproduced):
   * key padding (BERT-shaped case): after V,
     ``kv_len = torch.randint(kv_lo, kv_hi + 1, (B,))`` from the same generator;
   * default seed: the workload's index (1..5).
+
+Beyond the five square workloads: `DECODE_WORKLOADS` (one query row per head
+against a long key/value cache, for the split-KV path) with `make_qkv` (separate
+query and key counts); `make_bwd_inputs` (Q, K, V, then the output gradient dO,
+for the backward); `make_fp8_inputs` (the same N(0,1) draws quantized per tensor
+to e4m3 by torch's float8 conversion, for the e4m3 forward). Each keeps the
+draw order Q, K, V (then dO), then kv_len.
 """
 from __future__ import annotations
 
