@@ -78,8 +78,9 @@
 // and p_full phases, where n_t is the tile's number of key tiles (an idle
 // tile still takes part in its once-per-unit hand-offs), so every role can
 // compute every phase index and no barrier runs two phases ahead of a waiter.
-// (With one query tile the epilogue may find o_done two phases short of the
-// unit's last, so it waits for the last two phases in turn.)
+// (With one query tile and one accumulator the epilogue could find o_done one
+// phase short of, or one phase past, the unit's last; the second-last phase is
+// therefore waited for inside the last tile, before its P is handed over.)
 #pragma once
 
 #include <cuda_bf16.h>
@@ -721,6 +722,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int j_first = kDual ? wg : 0, j_step = kDual ? 2 : 1;
             const int n_own = kDual ? (n > wg ? (n - wg + 1) / 2 : 0) : n;
 
+            // One query tile with one accumulator: the last score tile was issued
+            // after P.V(n-3) only, so when the epilogue starts o_done may be one
+            // phase short of P.V(n-2) -- or, if P.V(n-1) has already finished,
+            // one phase past the last, with the same parity as phase n-2. The
+            // wait for phase n-2 is therefore made inside the last tile, before
+            // its P is handed over: P.V(n-1) cannot have been issued yet, so
+            // o_done is at phase n-2 or n-1 and the parity test is exact. The
+            // epilogue then waits for phase n-1 alone (o_done is at n-1 or n).
+            auto wait_second_last = [&](int j) -> bool {
+                if constexpr (!kDual && C::kQT == 1) {
+                    if (j == n - 1 && n >= 2) {
+                        bool w = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(n - 2)) & 1u, wd);
+                        return __all_sync(0xffffffffu, w);
+                    }
+                }
+                return true;
+            };
+
             for (int j = j_first; j < n; j += j_step) {
                 const int jo = kDual ? (j - wg) / 2 : j;       // index among this warpgroup's tiles
                 const int sb = (C::kQT == 2) ? t : (j & 1);   // this tile's S buffer
@@ -730,6 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 if (idle_warp) {
+                    ok = wait_second_last(j);
+                    if (!ok) break;
                     mbar_arrive(&bars->p_full[sb]);
                     continue;
                 }
@@ -795,6 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_wait_st();
                 tc_fence_before();
+                ok = wait_second_last(j);
+                if (!ok) break;
                 mbar_arrive(&bars->p_full[sb]);
             }
             if (!ok) break;
@@ -803,14 +826,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the unit's last o_done phase for this accumulator (its idle phase if none)
             const uint32_t last = o_base + (uint32_t)(n_own > 0 ? n_own - 1 : 0);
             o_base += (uint32_t)(n_own > 0 ? n_own : 1);
-            if (!kDual && C::kQT == 1 && n >= 2) {
-                // With one query tile the last score tile was issued after
-                // P.V(n-3) only, so o_done may still be in phase n-2: a parity
-                // wait for phase n-1 alone would pass at once. Wait in order.
-                ok = mbar_wait(&bars->o_done[t], (last - 1u) & 1u, wd);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-            }
             ok = mbar_wait(&bars->o_done[ob], last & 1u, wd);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
