@@ -49,20 +49,6 @@ def _bind(lib):
     i32p = ctypes.POINTER(ctypes.c_int32)
     u16p = ctypes.POINTER(ctypes.c_uint16)
     c_int, c_double = ctypes.c_int, ctypes.c_double
-    lib.oracle_attn_f64.argtypes = [dp, dp, dp, dp, dp, c_int, c_int, c_int,
-                                    c_int, c_double, c_int, i32p, c_int]
-    lib.oracle_attn_f64.restype = c_int
-    lib.oracle_attn_bf16.argtypes = [u16p, u16p, u16p, dp, dp, c_int, c_int,
-                                     c_int, c_int, c_double, c_int, i32p, i32p,
-                                     c_int, c_int]
-    lib.oracle_attn_bf16.restype = c_int
-    lib.oracle_attn_gqa_f64.argtypes = [dp, dp, dp, dp, dp, c_int, c_int, c_int, c_int,
-                                        c_int, c_double, c_int, i32p, c_int]
-    lib.oracle_attn_gqa_f64.restype = c_int
-    lib.oracle_attn_gqa_bf16.argtypes = [u16p, u16p, u16p, dp, dp, c_int, c_int, c_int,
-                                         c_int, c_int, c_double, c_int, i32p, i32p, c_int,
-                                         c_int]
-    lib.oracle_attn_gqa_bf16.restype = c_int
     lib.oracle_attn_general.argtypes = [dp, dp, dp, u16p, u16p, u16p, dp, dp, c_int, c_int,
                                          c_int, c_int, c_int, c_int, c_double, c_int, i32p,
                                          i32p, c_int, c_int]

@@ -205,51 +205,9 @@ static int attn_driver(const double *qd, const double *kd, const double *vd,
     return err;
 }
 
-/* fp64 inputs, all rows. q,k,v: [B,H,N,d]; o: [B,H,N,d]; lse: [B,H,N]. */
-int oracle_attn_f64(const double *q, const double *k, const double *v,
-                    double *o, double *lse, int B, int H, int N, int d,
-                    double scale, int causal, const int32_t *kv_len,
-                    int nthreads)
-{
-    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, H, N, N, d, scale,
-                       causal, kv_len, NULL, N, nthreads);
-}
-
-/* bf16 bit-pattern inputs; optional row subset (rows may be NULL => nrows == N). */
-int oracle_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                     double *o, double *lse, int B, int H, int N, int d,
-                     double scale, int causal, const int32_t *kv_len,
-                     const int32_t *rows, int nrows, int nthreads)
-{
-    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, H, N, N, d, scale,
-                       causal, kv_len, rows, nrows, nthreads);
-}
-
-/* Grouped/multi-query forms: q, o [B,H,N,d]; k, v [B,Hkv,N,d]. */
-int oracle_attn_gqa_f64(const double *q, const double *k, const double *v,
-                        double *o, double *lse, int B, int H, int Hkv, int N, int d,
-                        double scale, int causal, const int32_t *kv_len, int nthreads)
-{
-    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(q, k, v, NULL, NULL, NULL, o, lse, B, H, Hkv, N, N, d, scale,
-                       causal, kv_len, NULL, N, nthreads);
-}
-
-int oracle_attn_gqa_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                         double *o, double *lse, int B, int H, int Hkv, int N, int d,
-                         double scale, int causal, const int32_t *kv_len,
-                         const int32_t *rows, int nrows, int nthreads)
-{
-    if (!q || !k || !v || !o || !lse) return ORACLE_EINVAL;
-    return attn_driver(NULL, NULL, NULL, q, k, v, o, lse, B, H, Hkv, N, N, d, scale,
-                       causal, kv_len, rows, nrows, nthreads);
-}
-
 /* General form: q, o [B,H,Nq,d]; k, v [B,Hkv,Nk,d], Nq <= Nk (query row i at
  * key position i + Nk - Nq). Either fp64 inputs (qd/kd/vd) or bf16 bits
- * (qb/kb/vb); rows (nullable) as in oracle_attn_bf16, indices into Nq. */
+ * (qb/kb/vb); rows (nullable) as in attn_driver, indices into Nq. */
 int oracle_attn_general(const double *qd, const double *kd, const double *vd,
                         const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
                         double *o, double *lse, int B, int H, int Hkv, int Nq, int Nk,
