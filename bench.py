@@ -7,9 +7,11 @@
 A step is one full forward (one kernel launch) over the workload's tensors,
 which are resident in device memory before the timed region starts. The
 default workload is the long-context causal case (B=1, H=32, N=16384, d=128),
-the largest configuration; its inputs (3 x 128 MiB) exceed the 126 MB L2, so
-no L2 flush is done between steps. Metric: counted FLOPs 4*B*H*N^2*d (half
-when causal) per second, in TFLOP/s.
+the largest configuration; its inputs (3 x 128 MiB) exceed the 126 MB L2 by more
+than half again, so no L2 flush is done between steps. A workload whose inputs are
+smaller is timed with a 256 MiB buffer written before each step, and each step
+is timed alone. Metric: counted FLOPs 4*B*H*N^2*d (half when causal) per second,
+in TFLOP/s.
 
 With N > 1 GPUs (torchrun, one process per GPU) every rank runs its own
 replica of the workload (own seed): there is no data exchange on the path,
@@ -53,6 +55,58 @@ KERNEL_SOURCES = ["io_aware_exact_18_b200/csrc/fa_fwd_kernel.cuh",
 
 
 # ----------------------------------------------------------------- helpers
+L2_BYTES = 126 * 10**6          # B200 L2 cache
+FLUSH_BYTES = 256 * 2**20        # written before each timed step when inputs are small
+
+
+def l2_policy(input_bytes: int):
+    """Whether the timed steps flush the L2, and the line that says so.
+
+    Inputs of at least 1.5 x the 126 MB L2 stand for a cold cache by themselves
+    (a step cannot find most of them still cached from the step before); smaller
+    ones are timed with a 256 MiB buffer written before every step, each step
+    timed alone by its own pair of events."""
+    mib = input_bytes / 2**20
+    if input_bytes >= 1.5 * L2_BYTES:
+        return False, f"no flush: the step's inputs ({mib:.0f} MiB) exceed 1.5 x the 126 MB L2"
+    return True, (f"flush: the step's inputs ({mib:.0f} MiB) are under 1.5 x the 126 MB L2, "
+                  f"so a {FLUSH_BYTES >> 20} MiB buffer is written before each timed step, "
+                  "which is timed alone")
+
+
+def tensor_bytes(*xs) -> int:
+    return sum(x.numel() * x.element_size() for x in xs)
+
+
+def time_steps(torch, stream, step, steps: int, flush_buf=None) -> float:
+    """Device time of one step in ms, from CUDA events on the launching stream.
+    Without a flush buffer one pair of events brackets all the steps; with one,
+    the buffer is overwritten before every step and each step has its own pair,
+    so the flush is not timed."""
+    if flush_buf is None:
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(steps):
+                step()
+        ev1.record(stream)
+        stream.synchronize()
+        return ev0.elapsed_time(ev1) / steps
+    pairs = []
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush_buf.fill_(i & 0xFF)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            pairs.append((a, b))
+    stream.synchronize()
+    return sum(a.elapsed_time(b) for a, b in pairs) / steps
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -332,17 +386,14 @@ def our_arm(args, w):
         raise fa.FAError(st, "warm-up")
 
     # ---- timed region: device events on the launching stream
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    step_inputs = (qd, kd, vd) if kvd is None else (qd, kd, vd, kvd)
+    flush, l2_note = l2_policy(tensor_bytes(*step_inputs))
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    ev0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            step()
-    ev1.record(stream)
+    ms_local = time_steps(torch, stream, step, args.steps, flush_buf)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     if world > 1:
@@ -351,7 +402,6 @@ def our_arm(args, w):
     st = fa.fa_last_device_error(sh)
     if st != fa.FA_OK:
         raise fa.FAError(st, "timed region")
-    ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms_local, world)
     flops = w.flops()
     value = world * flops / (ms * 1e-3) / 1e12
@@ -437,8 +487,7 @@ def our_arm(args, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {**w.describe(), "parallelism": f"replicas x{world}",
-                       "l2": "no flush: inputs (3 x {:.0f} MiB) exceed the 126 MB L2".format(
-                           w.B * w.H * w.N * w.d * 2 / 2**20)},
+                       "l2": l2_note},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "clocks": clocks,
@@ -499,17 +548,14 @@ def decode_arm(args, w):
         for _ in range(args.warmup):
             step()
     stream.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    step_inputs = (qd, kd, vd)
+    flush, l2_note = l2_policy(tensor_bytes(*step_inputs))
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    ev0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            step()
-    ev1.record(stream)
+    ms_local = time_steps(torch, stream, step, args.steps, flush_buf)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     if world > 1:
@@ -518,7 +564,6 @@ def decode_arm(args, w):
     st = fa.fa_last_device_error(sh)
     if st != fa.FA_OK:
         raise fa.FAError(st, "timed region")
-    ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms_local, world)
     nbytes = w.algorithmic_bytes()
     value = world * nbytes / (ms * 1e-3) / 1e9
@@ -584,8 +629,7 @@ def decode_arm(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**w.describe(), "num_splits": splits,
                        "parallelism": f"replicas x{world}",
-                       "l2": "no flush: the K/V cache ({:.0f} MiB) exceeds the 126 MB L2".format(
-                           2 * w.B * w.H_kv * w.Nk * w.d * 2 / 2**20)},
+                       "l2": l2_note},
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -649,17 +693,14 @@ def backward_arm(args, w):
         for _ in range(args.warmup):
             step()
     stream.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    step_inputs = (qd, kd, vd, o, lse, dod)
+    flush, l2_note = l2_policy(tensor_bytes(*step_inputs))
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    ev0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            step()
-    ev1.record(stream)
+    ms_local = time_steps(torch, stream, step, args.steps, flush_buf)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     if world > 1:
@@ -668,7 +709,6 @@ def backward_arm(args, w):
     st = fa.fa_last_device_error(sh)
     if st != fa.FA_OK:
         raise fa.FAError(st, "timed region")
-    ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms_local, world)
     flops = 2.5 * w.flops()
     value = world * flops / (ms * 1e-3) / 1e12
@@ -736,8 +776,7 @@ def backward_arm(args, w):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**w.describe(), "pass": "backward", "parallelism": f"replicas x{world}",
-                       "l2": "no flush: Q, K, V, O, dO ({:.0f} MiB each) exceed the 126 MB L2"
-                       .format(w.B * w.H * w.N * w.d * 2 / 2**20)},
+                       "l2": l2_note},
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -793,17 +832,14 @@ def fp8_arm(args, w):
         for _ in range(args.warmup):
             step()
     stream.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    step_inputs = (qd, kd, vd)
+    flush, l2_note = l2_policy(tensor_bytes(*step_inputs))
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    ev0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            step()
-    ev1.record(stream)
+    ms_local = time_steps(torch, stream, step, args.steps, flush_buf)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     if world > 1:
@@ -812,7 +848,6 @@ def fp8_arm(args, w):
     st = fa.fa_last_device_error(sh)
     if st != fa.FA_OK:
         raise fa.FAError(st, "timed region")
-    ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms_local, world)
     flops = w.flops()
     value = world * flops / (ms * 1e-3) / 1e12
@@ -875,8 +910,7 @@ def fp8_arm(args, w):
             "dtype": "e4m3", "data": "synthetic",
             "config": {**w.describe(), "inputs": "e4m3, per-tensor descale amax/448",
                        "parallelism": f"replicas x{world}",
-                       "l2": "no flush: inputs (3 x {:.0f} MiB) exceed the 126 MB L2".format(
-                           w.B * w.H * w.N * w.d / 2**20)},
+                       "l2": l2_note},
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},

@@ -52,3 +52,89 @@ def test_missing_extension_fails_loudly(tmp_path):
     import io_aware_exact_18_b200 as fa
     with pytest.raises(ImportError):
         fa.load_library(os.path.join(str(tmp_path), "libfa.so"))
+
+
+def _input_bytes(w):
+    kv = w.kv_heads
+    return 2 * w.B * w.N * w.d * (w.H + 2 * kv)
+
+
+def test_l2_policy_flushes_the_workloads_that_fit_near_the_l2():
+    for idx in (1, 2, 3, 4):
+        flush, note = bench.l2_policy(_input_bytes(workloads.get(idx)))
+        assert flush and note.startswith("flush:")
+    flush, note = bench.l2_policy(_input_bytes(workloads.get(5)))
+    assert not flush and note.startswith("no flush:") and "384 MiB" in note
+    for dw in workloads.DECODE_WORKLOADS:
+        kv_bytes = 2 * 2 * dw.B * dw.H_kv * dw.Nk * dw.d
+        assert not bench.l2_policy(kv_bytes)[0]
+    assert bench.FLUSH_BYTES > 2 * bench.L2_BYTES
+    assert bench.l2_policy(int(1.5 * bench.L2_BYTES))[0] is False
+    assert bench.l2_policy(int(1.5 * bench.L2_BYTES) - 1)[0] is True
+
+
+class _FakeCuda:
+    """Stands in for torch.cuda in time_steps: records the order of events,
+    steps and flushes, and gives each event pair a fixed duration."""
+
+    def __init__(self, log):
+        self.log = log
+        cuda = self
+
+        class Event:
+            n = 0
+
+            def __init__(self, enable_timing=False):
+                assert enable_timing
+                Event.n += 1
+                self.id = Event.n
+
+            def record(self, stream):
+                cuda.log.append(("record", self.id))
+
+            def elapsed_time(self, other):
+                return 2.0 * (other.id - self.id)
+
+        self.Event = Event
+
+    class _Ctx:
+        def __enter__(self):
+            return self
+
+        def __exit__(self, *a):
+            return False
+
+    def stream(self, s):
+        return self._Ctx()
+
+
+class _FakeStream:
+    def __init__(self, log):
+        self.log = log
+
+    def synchronize(self):
+        self.log.append(("sync",))
+
+
+class _FakeBuf:
+    def __init__(self, log):
+        self.log = log
+
+    def fill_(self, v):
+        self.log.append(("flush", v))
+
+
+def test_time_steps_flushes_before_each_step_and_times_only_the_step():
+    log = []
+    fake_torch = type("T", (), {})()
+    fake_torch.cuda = _FakeCuda(log)
+    step = lambda: log.append(("step",))  # noqa: E731
+    ms = bench.time_steps(fake_torch, _FakeStream(log), step, 3, _FakeBuf(log))
+    kinds = [e[0] for e in log]
+    assert kinds == ["flush", "record", "step", "record"] * 3 + ["sync"]
+    assert ms == pytest.approx(2.0)   # each pair is consecutive events: 2.0 ms apiece
+
+    log.clear()
+    ms = bench.time_steps(fake_torch, _FakeStream(log), step, 4, None)
+    assert [e[0] for e in log] == ["record"] + ["step"] * 4 + ["record", "sync"]
+    assert ms == pytest.approx(2.0 / 4)
