@@ -13,6 +13,9 @@ Two independent routes to the same result:
   fp64 C. The pages state no backward algorithm; this is the exact gradient.
 * :func:`attention_bwd_dq_rows` -- dQ of selected query rows only (the same
   definition; dQ row i depends on row i alone), for checks at full size.
+* :func:`attention_bwd_kv_rows` -- dK and dV of selected key rows only (the
+  same definition, every query row's softmax still taken in full), for
+  checks at full size.
 * :mod:`oracle.fp8` -- e4m3 decoding by the format's definition, feeding the
   fp64 attention of the dequantized tensors.
 * :func:`online.attention_online` -- a blockwise online-softmax evaluation in
@@ -60,6 +63,10 @@ def _bind(lib):
                                             c_int, c_int, c_double, c_int, i32p, i32p, c_int,
                                             c_int]
     lib.oracle_attn_bwd_dq_rows.restype = c_int
+    lib.oracle_attn_bwd_kv_rows.argtypes = [u16p, u16p, u16p, u16p, dp, dp, c_int, c_int, c_int,
+                                            c_int, c_int, c_double, c_int, i32p, i32p, c_int,
+                                            c_int]
+    lib.oracle_attn_bwd_kv_rows.restype = c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     return lib
@@ -229,3 +236,39 @@ def attention_bwd_dq_rows(q, k, v, do, scale, rows, causal=False, kv_len=None, n
     if rc != 0:
         raise RuntimeError(f"oracle returned error {rc}")
     return out
+
+
+def attention_bwd_kv_rows(q, k, v, do, scale, rows, causal=False, kv_len=None, nthreads=0,
+                          lib=None):
+    """dK and dV of the given key rows of every (b, K/V head), in fp64: two
+    arrays [B, Hkv, len(rows), d]. Same definition as attention_bwd (each
+    query row's softmax and D_i are computed over all its keys; only the sums
+    into dK and dV are restricted to the selected keys); bf16 torch tensors
+    or uint16 arrays, square (Nq == Nk)."""
+    lib = lib or load()
+    arrs = [_as_numpy(x) for x in (q, k, v, do)]
+    if not all(b for _, b in arrs):
+        raise TypeError("q, k, v, do must be bf16")
+    (qa, _), (ka, _), (va, _), (da, _) = arrs
+    B, H, N, d = qa.shape
+    Hkv = ka.shape[1]
+    if ka.shape != (B, Hkv, N, d) or va.shape != ka.shape or da.shape != qa.shape:
+        raise ValueError("bad shapes")
+    ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    kvp = None
+    if kv_len is not None:
+        kvl = np.ascontiguousarray(np.asarray(
+            kv_len.cpu().numpy() if hasattr(kv_len, "cpu") else kv_len, dtype=np.int32))
+        kvp = kvl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    dk = np.zeros((B, Hkv, len(ra), d), dtype=np.float64)
+    dv = np.zeros((B, Hkv, len(ra), d), dtype=np.float64)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    dp = ctypes.POINTER(ctypes.c_double)
+    rc = lib.oracle_attn_bwd_kv_rows(*(a.ctypes.data_as(u16p) for a in (qa, ka, va, da)),
+                                     dk.ctypes.data_as(dp), dv.ctypes.data_as(dp), B, H, Hkv, N,
+                                     d, float(scale), int(bool(causal)), kvp,
+                                     ra.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                     len(ra), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle returned error {rc}")
+    return dk, dv

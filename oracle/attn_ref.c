@@ -238,9 +238,14 @@ int oracle_attn_general(const double *qd, const double *kd, const double *vd,
  * q, dO, dq: [B,H,N,d]; k, v, dk, dv: [B,Hkv,N,d] (square: Nq == Nk == N).
  * Inputs fp64 (qd..dod) or bf16 bits (qb..dob), exactly one set non-null.
  */
-static void bwd_one_row(const double *qi, const double *doi, const double *K, const double *V,
-                        int N, int d, double scale, int i, int causal, int kv_lim,
-                        double *prow, double *dsrow, double *dqi, double *dK, double *dV)
+/*
+ * Row i's softmax weights P_ij (0 for hidden keys) into prow, dP_ij =
+ * <dO_i, v_j> into dprow (0 where P_ij = 0), and D_i = sum_j P_ij dP_ij as the
+ * return value. Returns 0 with prow and dprow all 0 if row i sees no key.
+ */
+static double bwd_row_p_dp(const double *qi, const double *doi, const double *K,
+                           const double *V, int N, int d, double scale, int i, int causal,
+                           int kv_lim, double *prow, double *dprow)
 {
     double m = -INFINITY;
     for (int j = 0; j < N; ++j) {
@@ -254,30 +259,40 @@ static void bwd_one_row(const double *qi, const double *doi, const double *K, co
         prow[j] = scale * dot;
         if (prow[j] > m) m = prow[j];
     }
-    for (int t = 0; t < d; ++t) dqi[t] = 0.0;
-    if (m == -INFINITY) return;
+    if (m == -INFINITY) {
+        for (int j = 0; j < N; ++j) prow[j] = dprow[j] = 0.0;
+        return 0.0;
+    }
     double sum = 0.0;
     for (int j = 0; j < N; ++j)
         if (prow[j] != -INFINITY) sum += exp(prow[j] - m);
     for (int j = 0; j < N; ++j)
         prow[j] = (prow[j] == -INFINITY) ? 0.0 : exp(prow[j] - m) / sum;
-    /* dP_ij and D_i */
     double D = 0.0;
     for (int j = 0; j < N; ++j) {
         if (prow[j] == 0.0) {
-            dsrow[j] = 0.0;
+            dprow[j] = 0.0;
             continue;
         }
         const double *vrow = V + (size_t)j * d;
         double dot = 0.0;
         for (int t = 0; t < d; ++t) dot += doi[t] * vrow[t];
-        dsrow[j] = dot;
+        dprow[j] = dot;
         D += prow[j] * dot;
     }
+    return D;
+}
+
+static void bwd_one_row(const double *qi, const double *doi, const double *K, const double *V,
+                        int N, int d, double scale, int i, int causal, int kv_lim,
+                        double *prow, double *dprow, double *dqi, double *dK, double *dV)
+{
+    const double D = bwd_row_p_dp(qi, doi, K, V, N, d, scale, i, causal, kv_lim, prow, dprow);
+    for (int t = 0; t < d; ++t) dqi[t] = 0.0;
     for (int j = 0; j < N; ++j) {
         const double pij = prow[j];
         if (pij == 0.0) continue;
-        const double ds = pij * (dsrow[j] - D);
+        const double ds = pij * (dprow[j] - D);
         const double *krow = K + (size_t)j * d;
         double *dkj = dK + (size_t)j * d;
         double *dvj = dV + (size_t)j * d;
@@ -326,7 +341,7 @@ int oracle_attn_bwd(const double *qd, const double *kd, const double *vd, const 
             continue;
         }
         double *K = buf, *V = buf + head, *Q = buf + 2 * head, *dO = buf + 3 * head;
-        double *prow = buf + 4 * head, *dsrow = prow + N;
+        double *prow = buf + 4 * head, *dprow = prow + N;
         const size_t kvbase = (size_t)g * head;
         for (size_t e = 0; e < head; ++e) {
             K[e] = bits ? bf16_to_f64(kb[kvbase + e]) : kd[kvbase + e];
@@ -342,7 +357,7 @@ int oracle_attn_bwd(const double *qd, const double *kd, const double *vd, const 
             }
             for (int i = 0; i < N; ++i)
                 bwd_one_row(Q + (size_t)i * d, dO + (size_t)i * d, K, V, N, d, scale, i, causal,
-                            kv_lim, prow, dsrow, dq + qbase + (size_t)i * d, dK, dV);
+                            kv_lim, prow, dprow, dq + qbase + (size_t)i * d, dK, dV);
         }
         free(buf);
     }
@@ -384,7 +399,7 @@ int oracle_attn_bwd_dq_rows(const uint16_t *qb, const uint16_t *kb, const uint16
         } else {
             double *K = buf, *V = buf + head, *dKs = buf + 2 * head, *dVs = buf + 3 * head;
             double *qi = buf + 4 * head, *doi = qi + d;
-            double *prow = doi + 2 * (size_t)d, *dsrow = prow + N;
+            double *prow = doi + 2 * (size_t)d, *dprow = prow + N;
             int loaded = -1;
 #pragma omp for schedule(dynamic, 1)
             for (int bh = 0; bh < B * H; ++bh) {
@@ -411,13 +426,104 @@ int oracle_attn_bwd_dq_rows(const uint16_t *qb, const uint16_t *kb, const uint16
                         doi[t] = bf16_to_f64(dob[qoff + t]);
                     }
                     for (size_t e = 0; e < head; ++e) dKs[e] = dVs[e] = 0.0;
-                    bwd_one_row(qi, doi, K, V, N, d, scale, i, causal, kv_lim, prow, dsrow,
+                    bwd_one_row(qi, doi, K, V, N, d, scale, i, causal, kv_lim, prow, dprow,
                                 dq_rows + ((size_t)bh * nrows + r) * d, dKs, dVs);
                 }
             }
             free(buf);
         }
     }
+    return err;
+}
+
+/*
+ * dK and dV of selected key rows only (same definition as oracle_attn_bwd:
+ * dK_j = scale sum_i dS_ij q_i and dV_j = sum_i P_ij dO_i over every query
+ * row i of every query head of the K/V head's group). Key row j needs P_ij,
+ * dP_ij and D_i of every row i, so each row's softmax and D are still
+ * computed in full; only the accumulation is restricted to the selected keys.
+ * For checks at sizes where the full backward is out of reach. dk_rows,
+ * dv_rows: [B,Hkv,nrows,d]. bf16 inputs only.
+ */
+int oracle_attn_bwd_kv_rows(const uint16_t *qb, const uint16_t *kb, const uint16_t *vb,
+                            const uint16_t *dob, double *dk_rows, double *dv_rows, int B, int H,
+                            int Hkv, int N, int d, double scale, int causal,
+                            const int32_t *kv_len, const int32_t *rows, int nrows, int nthreads)
+{
+    if (!qb || !kb || !vb || !dob || !dk_rows || !dv_rows || !rows) return ORACLE_EINVAL;
+    int rc = check_args(B, H, N, d, scale, causal);
+    if (rc) return rc;
+    if (B == 0 || H == 0 || N == 0 || nrows == 0) return ORACLE_OK;
+    if (Hkv <= 0 || Hkv > H || H % Hkv != 0 || nrows < 0) return ORACLE_EINVAL;
+    for (int r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= N) return ORACLE_EINVAL;
+    const int G = H / Hkv;
+    const size_t head = (size_t)N * d, sel = (size_t)nrows * d;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    double *K = (double *)malloc(4 * head * sizeof(double));
+    if (!K) return ORACLE_ENOMEM;
+    double *V = K + head, *Q = K + 2 * head, *dO = K + 3 * head;
+    int err = ORACLE_OK;
+    for (int g = 0; g < B * Hkv && err == ORACLE_OK; ++g) {
+        const int b = g / Hkv, hk = g % Hkv;
+        int kv_lim = N;
+        if (kv_len) {
+            kv_lim = kv_len[b];
+            if (kv_lim < 0) kv_lim = 0;
+            if (kv_lim > N) kv_lim = N;
+        }
+        for (size_t e = 0; e < head; ++e) {
+            K[e] = bf16_to_f64(kb[(size_t)g * head + e]);
+            V[e] = bf16_to_f64(vb[(size_t)g * head + e]);
+        }
+        double *dKr = dk_rows + (size_t)g * sel, *dVr = dv_rows + (size_t)g * sel;
+        for (size_t e = 0; e < sel; ++e) dKr[e] = dVr[e] = 0.0;
+        for (int hq = hk * G; hq < (hk + 1) * G; ++hq) {
+            const size_t qbase = ((size_t)b * H + hq) * head;
+            for (size_t e = 0; e < head; ++e) {
+                Q[e] = bf16_to_f64(qb[qbase + e]);
+                dO[e] = bf16_to_f64(dob[qbase + e]);
+            }
+#pragma omp parallel
+            {
+                /* per thread: one row's P and dP, and private sums for the selected keys */
+                double *buf = (double *)malloc((2 * (size_t)N + 2 * sel) * sizeof(double));
+                if (!buf) {
+#pragma omp atomic write
+                    err = ORACLE_ENOMEM;
+                } else {
+                    double *prow = buf, *dprow = buf + N, *aK = buf + 2 * (size_t)N, *aV = aK + sel;
+                    for (size_t e = 0; e < 2 * sel; ++e) aK[e] = 0.0;
+#pragma omp for schedule(dynamic, 16)
+                    for (int i = 0; i < N; ++i) {
+                        const double *qi = Q + (size_t)i * d, *doi = dO + (size_t)i * d;
+                        const double D = bwd_row_p_dp(qi, doi, K, V, N, d, scale, i, causal,
+                                                      kv_lim, prow, dprow);
+                        for (int r = 0; r < nrows; ++r) {
+                            const double pij = prow[rows[r]];
+                            if (pij == 0.0) continue;
+                            const double ds = pij * (dprow[rows[r]] - D);
+                            for (int t = 0; t < d; ++t) {
+                                aK[(size_t)r * d + t] += scale * ds * qi[t];
+                                aV[(size_t)r * d + t] += pij * doi[t];
+                            }
+                        }
+                    }
+#pragma omp critical
+                    for (size_t e = 0; e < sel; ++e) {
+                        dKr[e] += aK[e];
+                        dVr[e] += aV[e];
+                    }
+                    free(buf);
+                }
+            }
+        }
+    }
+    free(K);
     return err;
 }
 

@@ -139,8 +139,29 @@ def pin_bwd_dq_rows_equal_full(lib):
         assert np.array_equal(part, full[:, :, rows]), (causal, kv_len)
 
 
+def pin_bwd_kv_rows_equal_full(lib):
+    """The key-row driver gives the full backward's dK and dV rows (to fp64
+    rounding: it sums the query rows in another order), with grouped heads,
+    causal and padding masks, and keys no row sees (all-zero rows)."""
+    import torch
+    g = torch.Generator().manual_seed(17)
+    q, do = (torch.randn(2, 4, 40, 8, generator=g).to(torch.bfloat16) for _ in range(2))
+    k, v = (torch.randn(2, 2, 40, 8, generator=g).to(torch.bfloat16) for _ in range(2))
+    rows = [0, 1, 13, 25, 38, 39]
+    for causal, kv_len in ((True, None), (False, [30, 40]), (True, [7, 40])):
+        _, dk, dv = _bwd(lib, q, k, v, do, 0.45, causal, kv_len)
+        pk, pv = oracle.attention_bwd_kv_rows(q, k, v, do, 0.45, rows, causal=causal,
+                                              kv_len=kv_len, nthreads=3, lib=lib)
+        for part, full in ((pk, dk[:, :, rows]), (pv, dv[:, :, rows])):
+            assert np.allclose(part, full, rtol=1e-12, atol=1e-13), (causal, kv_len)
+        if kv_len is not None:        # keys at or past kv_len: no row sees them
+            hidden = np.array(rows)[None, :] >= np.array(kv_len)[:, None]
+            assert np.all(pk[hidden.nonzero()[0], :, hidden.nonzero()[1]] == 0.0)
+
+
 PINS = [pin_bwd_finite_differences, pin_bwd_torch_autograd, pin_bwd_invariants,
-        pin_bwd_zero_output_gradient, pin_bwd_bf16_inputs_equal_f64, pin_bwd_dq_rows_equal_full]
+        pin_bwd_zero_output_gradient, pin_bwd_bf16_inputs_equal_f64, pin_bwd_dq_rows_equal_full,
+        pin_bwd_kv_rows_equal_full]
 
 
 def failures(lib):

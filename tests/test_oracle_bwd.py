@@ -11,8 +11,8 @@ from tests import oracle_bwd_pins
 SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_ref.c")
 
 MUTANTS = {
-    "missing_D_term": ("const double ds = pij * (dsrow[j] - D);",
-                       "const double ds = pij * dsrow[j];"),
+    "missing_D_term": ("const double ds = pij * (dprow[j] - D);",
+                       "const double ds = pij * dprow[j];"),
     "D_sign_flipped": ("D += prow[j] * dot;", "D -= prow[j] * dot;"),
     "dK_missing_scale": ("dkj[t] += scale * ds * qi[t];", "dkj[t] += ds * qi[t];"),
     "dQ_missing_scale": ("dqi[t] += scale * ds * krow[t];", "dqi[t] += ds * krow[t];"),
@@ -21,11 +21,33 @@ MUTANTS = {
     "P_unnormalised": ("exp(prow[j] - m) / sum;", "exp(prow[j] - m);"),
     "dP_uses_key": ("dot += doi[t] * vrow[t];", "dot += doi[t] * K[(size_t)j * d + t];"),
     "group_sum_overwritten": (
-        "for (int hq = hk * G; hq < (hk + 1) * G; ++hq) {",
         "for (int hq = hk * G; hq < (hk + 1) * G; ++hq) {\n"
-        "            for (size_t e = 0; e < head; ++e) dK[e] = dV[e] = 0.0;"),
+        "            const size_t qbase = ((size_t)b * H + hq) * head;\n"
+        "            for (size_t e = 0; e < head; ++e) {\n"
+        "                Q[e] = bits ?",
+        "for (int hq = hk * G; hq < (hk + 1) * G; ++hq) {\n"
+        "            for (size_t e = 0; e < head; ++e) dK[e] = dV[e] = 0.0;\n"
+        "            const size_t qbase = ((size_t)b * H + hq) * head;\n"
+        "            for (size_t e = 0; e < head; ++e) {\n"
+        "                Q[e] = bits ?"),
     "backward_mask_not_causal": ("if (!key_allowed(i, j, causal, kv_lim, 0)) {",
                                  "if (!key_allowed(i, j, 0, kv_lim, 0)) {"),
+    "kv_rows_dK_missing_scale": ("aK[(size_t)r * d + t] += scale * ds * qi[t];",
+                                 "aK[(size_t)r * d + t] += ds * qi[t];"),
+    "kv_rows_dV_uses_dS": ("aV[(size_t)r * d + t] += pij * doi[t];",
+                           "aV[(size_t)r * d + t] += ds * doi[t];"),
+    "kv_rows_one_head_of_group": ("for (int hq = hk * G; hq < (hk + 1) * G; ++hq) {\n"
+                                  "            const size_t qbase = ((size_t)b * H + hq) * head;\n"
+                                  "            for (size_t e = 0; e < head; ++e) {\n"
+                                  "                Q[e] = bf16_to_f64(qb[qbase + e]);\n"
+                                  "                dO[e] = bf16_to_f64(dob[qbase + e]);\n"
+                                  "            }\n#pragma omp parallel",
+                                  "for (int hq = hk * G; hq < hk * G + 1; ++hq) {\n"
+                                  "            const size_t qbase = ((size_t)b * H + hq) * head;\n"
+                                  "            for (size_t e = 0; e < head; ++e) {\n"
+                                  "                Q[e] = bf16_to_f64(qb[qbase + e]);\n"
+                                  "                dO[e] = bf16_to_f64(dob[qbase + e]);\n"
+                                  "            }\n#pragma omp parallel"),
 }
 
 
