@@ -78,11 +78,14 @@ def tensor_bytes(*xs) -> int:
     return sum(x.numel() * x.element_size() for x in xs)
 
 
-def time_steps(torch, stream, step, steps: int, flush_buf=None) -> float:
+def time_steps(torch, stream, step, steps: int, flush_buf=None, clean_buf=None) -> float:
     """Device time of one step in ms, from CUDA events on the launching stream.
     Without a flush buffer one pair of events brackets all the steps; with one,
     the buffer is overwritten before every step and each step has its own pair,
-    so the flush is not timed."""
+    so the flush is not timed. With clean_buf as well, that second buffer is
+    read after the write (a max-reduction), so the L2 the step starts with
+    holds clean lines of it instead of the first buffer's dirty ones, and the
+    step's first reads do not wait behind their write-back."""
     if flush_buf is None:
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
@@ -97,6 +100,8 @@ def time_steps(torch, stream, step, steps: int, flush_buf=None) -> float:
     with torch.cuda.stream(stream):
         for i in range(steps):
             flush_buf.fill_(i & 0xFF)
+            if clean_buf is not None:
+                clean_buf.max()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -131,21 +136,25 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(workload_name: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; otherwise None."""
+    """DRAM bytes per launch from the committed ncu record, if it was taken on
+    the current kernel sources: {"read": R, "write": W, "case": ...}, else
+    None. Writes that are still dirty in L2 when the kernel ends are not in W
+    (they reach DRAM later), so W can sit below the O + lse bytes."""
     path = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
     if not os.path.exists(path):
         return None
     vals = {}
     with open(path) as f:
         for line in f:
-            if ":" in line:
+            if ":" in line and not line.startswith("#"):
                 key, val = line.split(":", 1)
                 vals[key.strip()] = val.strip()
     if vals.get("kernel_source_sha256_16") != kernel_source_hash():
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
+        return {"read": float(vals["dram_read_bytes_per_launch"]),
+                "write": float(vals["dram_write_bytes_per_launch"]),
+                "case": vals.get("measured_case", "")}
     except (KeyError, ValueError):
         return None
 
@@ -332,6 +341,69 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def square_call(fa, w, qd, kd, vd, od, lsed, kvd, sh):
+    """One forward launch of a square workload through the C ABI."""
+    if w.kv_heads != w.H:
+        st = fa.fa_fwd_gqa(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                           lsed.data_ptr(), w.B, w.H, w.kv_heads, w.N, w.d, w.scale,
+                           int(w.causal), None if kvd is None else kvd.data_ptr(), sh)
+    elif kvd is None:
+        st = fa.fa_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                       lsed.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal), sh)
+    else:
+        st = fa.fa_fwd_kvlen(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                             lsed.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal),
+                             kvd.data_ptr(), sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "fa_fwd")
+
+
+def time_workload(torch, fa, w, dev, stream, steps, warmup, seed, clean_buf=None):
+    """Device time of one forward launch of workload w (ms), with its inputs
+    resident in HBM and the L2 policy of l2_policy; returns (ms, l2 note,
+    ms after a clean flush or None). The clean-flush time is taken only for a
+    workload that is flushed at all, and only when clean_buf is given."""
+    q, k, v, kv_len = workloads.make_inputs(w, seed=seed)
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    kvd = None if kv_len is None else kv_len.to(dev)
+    od = torch.empty_like(qd)
+    lsed = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    sh = stream.cuda_stream
+
+    def step():
+        square_call(fa, w, qd, kd, vd, od, lsed, kvd, sh)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    stream.synchronize()
+    step_inputs = (qd, kd, vd) if kvd is None else (qd, kd, vd, kvd)
+    flush, l2_note = l2_policy(tensor_bytes(*step_inputs))
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
+    ms = time_steps(torch, stream, step, steps, flush_buf)
+    ms_clean = None
+    if flush and clean_buf is not None:
+        ms_clean = time_steps(torch, stream, step, steps, flush_buf, clean_buf)
+    st = fa.fa_last_device_error(sh)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, f"timed region of {w.name}")
+    return ms, l2_note, ms_clean
+
+
+def config_entry(w, ms, world, peak, l2_note, ms_clean=None):
+    tflops = world * w.flops() / (ms * 1e-3) / 1e12
+    e = {"workload": w.name, "ms_per_launch": ms, "tflops": tflops,
+         "frac_of_measured_peak": tflops / world / peak, "l2": l2_note}
+    if ms_clean is not None:
+        tc = world * w.flops() / (ms_clean * 1e-3) / 1e12
+        e["clean_flush"] = {
+            "ms_per_launch": ms_clean, "tflops": tc, "frac_of_measured_peak": tc / world / peak,
+            "note": "the same launches after the 256 MiB write and then a read of a second "
+                    "256 MiB buffer: the inputs are still out of the L2, but the L2 holds no "
+                    "dirty lines whose write-back the first reads would wait behind"}
+    return e
+
+
 def our_arm(args, w):
     import datetime
 
@@ -361,19 +433,7 @@ def our_arm(args, w):
     sh = stream.cuda_stream
 
     def step():
-        if w.kv_heads != w.H:
-            st = fa.fa_fwd_gqa(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
-                               lsed.data_ptr(), w.B, w.H, w.kv_heads, w.N, w.d, w.scale,
-                               int(w.causal), None if kvd is None else kvd.data_ptr(), sh)
-        elif kvd is None:
-            st = fa.fa_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
-                           lsed.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal), sh)
-        else:
-            st = fa.fa_fwd_kvlen(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
-                                 lsed.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal),
-                                 kvd.data_ptr(), sh)
-        if st != fa.FA_OK:
-            raise fa.FAError(st, "fa_fwd")
+        square_call(fa, w, qd, kd, vd, od, lsed, kvd, sh)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -455,16 +515,24 @@ def our_arm(args, w):
     peaks, peak_src = load_peaks()
     achieved = flops / (ms_local * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = recorded_traffic(w.name)
+    rec = recorded_traffic(w.name)
+    alg_read = float(w.B * w.N * (w.H + 2 * w.kv_heads) * w.d * 2)      # Q, K, V once
+    alg_write = float(w.B * w.N * w.H * (w.d * 2 + 4))                   # O, lse once
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
+                "frac": achieved / peak,
+                "traffic": None if rec is None else rec["read"] + rec["write"],
                 "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
                 "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                 "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
-                "algorithmic_bytes": float(w.B * w.N * (2 * w.H * w.d * 2 + 2 * w.kv_heads * w.d * 2
-                                                        + 4 * w.H)),
-                "traffic_over_algorithmic": (None if traffic is None else traffic / float(
-                    w.B * w.N * (2 * w.H * w.d * 2 + 2 * w.kv_heads * w.d * 2 + 4 * w.H))),
+                "algorithmic_bytes": alg_read + alg_write,
+                "traffic_read": None if rec is None else rec["read"],
+                "traffic_write": None if rec is None else rec["write"],
+                "read_over_algorithmic": None if rec is None else rec["read"] / alg_read,
+                "write_over_algorithmic": None if rec is None else rec["write"] / alg_write,
+                "traffic_note": ("ncu dram__bytes_read.sum / dram__bytes_write.sum of one launch"
+                                 + ("" if rec is None else f" ({rec['case']})")
+                                 + "; reads are compared with Q + K + V, writes with O + lse; "
+                                 "writes still dirty in L2 when the kernel ends are not counted"),
                 # secondary bound: one exponential per visible score; MUFU ex2 runs 16 per
                 # clock per SM (148 SMs) at the sampled SM clock
                 "exp_per_s": vis / (ms_local * 1e-3),
@@ -472,6 +540,26 @@ def our_arm(args, w):
                     16 * 148 * float(clocks.get("sm_mhz") or 1965) * 1e6),
                 "effective_tflops_visible_keys": eff_flops / (ms_local * 1e-3) / 1e12,
                 "kernel": f"fa_fwd_sm100<{w.d},{1 if w.d == 256 else 2},square>"}
+
+    # ---- every square workload in this process, each under its own L2 policy
+    # (the headline workload's entry is the measurement above)
+    configs = None
+    if not args.no_configs and args.shape is None:
+        del qd, kd, vd, od, kvd, flush_buf
+        torch.cuda.empty_cache()
+        configs = []
+        clean_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        clean_buf.fill_(1)
+        for cw in workloads.WORKLOADS:
+            if cw.name == w.name:
+                configs.append(config_entry(cw, ms, world, peak, l2_note))
+                continue
+            cms, cnote, cclean = time_workload(torch, fa, cw, dev, stream, args.steps,
+                                               args.warmup, seed=cw.index + 1000 * rank,
+                                               clean_buf=clean_buf)
+            configs.append(config_entry(cw, max_over_ranks(cms, world), world, peak, cnote,
+                                        None if cclean is None else max_over_ranks(cclean, world)))
+        del clean_buf
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -494,6 +582,7 @@ def our_arm(args, w):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": args.steps,
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -936,6 +1025,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload timings of the five square workloads")
     ap.add_argument("--fp8", action="store_true",
                     help="time the e4m3 forward (fa_fwd_fp8) on the workload instead")
     ap.add_argument("--backward", action="store_true",

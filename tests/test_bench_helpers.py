@@ -40,10 +40,13 @@ def test_source_hash_ignores_comments(tmp_path, monkeypatch):
 def test_recorded_traffic_requires_matching_sources(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "traffic_x.txt").write_text("kernel_source_sha256_16: abc\ndram_bytes_per_launch: 123\n")
+    (prof / "traffic_x.txt").write_text(
+        "# comment: lines with a colon after a hash are ignored\n"
+        "kernel_source_sha256_16: abc\nmeasured_case: B1 H2\n"
+        "dram_read_bytes_per_launch: 100\ndram_write_bytes_per_launch: 23\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc")
-    assert bench.recorded_traffic("x") == 123.0
+    assert bench.recorded_traffic("x") == {"read": 100.0, "write": 23.0, "case": "B1 H2"}
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "def")
     assert bench.recorded_traffic("x") is None
 
