@@ -78,14 +78,11 @@ def tensor_bytes(*xs) -> int:
     return sum(x.numel() * x.element_size() for x in xs)
 
 
-def time_steps(torch, stream, step, steps: int, flush_buf=None, clean_buf=None) -> float:
+def time_steps(torch, stream, step, steps: int, flush_buf=None) -> float:
     """Device time of one step in ms, from CUDA events on the launching stream.
     Without a flush buffer one pair of events brackets all the steps; with one,
     the buffer is overwritten before every step and each step has its own pair,
-    so the flush is not timed. With clean_buf as well, that second buffer is
-    read after the write (a max-reduction), so the L2 the step starts with
-    holds clean lines of it instead of the first buffer's dirty ones, and the
-    step's first reads do not wait behind their write-back."""
+    so the flush is not timed."""
     if flush_buf is None:
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
@@ -100,8 +97,6 @@ def time_steps(torch, stream, step, steps: int, flush_buf=None, clean_buf=None) 
     with torch.cuda.stream(stream):
         for i in range(steps):
             flush_buf.fill_(i & 0xFF)
-            if clean_buf is not None:
-                clean_buf.max()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -358,11 +353,9 @@ def square_call(fa, w, qd, kd, vd, od, lsed, kvd, sh):
         raise fa.FAError(st, "fa_fwd")
 
 
-def time_workload(torch, fa, w, dev, stream, steps, warmup, seed, clean_buf=None):
+def time_workload(torch, fa, w, dev, stream, steps, warmup, seed):
     """Device time of one forward launch of workload w (ms), with its inputs
-    resident in HBM and the L2 policy of l2_policy; returns (ms, l2 note,
-    ms after a clean flush or None). The clean-flush time is taken only for a
-    workload that is flushed at all, and only when clean_buf is given."""
+    resident in HBM and the L2 policy of l2_policy; returns (ms, l2 note)."""
     q, k, v, kv_len = workloads.make_inputs(w, seed=seed)
     qd, kd, vd = (x.to(dev) for x in (q, k, v))
     kvd = None if kv_len is None else kv_len.to(dev)
@@ -381,27 +374,16 @@ def time_workload(torch, fa, w, dev, stream, steps, warmup, seed, clean_buf=None
     flush, l2_note = l2_policy(tensor_bytes(*step_inputs))
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
     ms = time_steps(torch, stream, step, steps, flush_buf)
-    ms_clean = None
-    if flush and clean_buf is not None:
-        ms_clean = time_steps(torch, stream, step, steps, flush_buf, clean_buf)
     st = fa.fa_last_device_error(sh)
     if st != fa.FA_OK:
         raise fa.FAError(st, f"timed region of {w.name}")
-    return ms, l2_note, ms_clean
+    return ms, l2_note
 
 
-def config_entry(w, ms, world, peak, l2_note, ms_clean=None):
+def config_entry(w, ms, world, peak, l2_note):
     tflops = world * w.flops() / (ms * 1e-3) / 1e12
-    e = {"workload": w.name, "ms_per_launch": ms, "tflops": tflops,
-         "frac_of_measured_peak": tflops / world / peak, "l2": l2_note}
-    if ms_clean is not None:
-        tc = world * w.flops() / (ms_clean * 1e-3) / 1e12
-        e["clean_flush"] = {
-            "ms_per_launch": ms_clean, "tflops": tc, "frac_of_measured_peak": tc / world / peak,
-            "note": "the same launches after the 256 MiB write and then a read of a second "
-                    "256 MiB buffer: the inputs are still out of the L2, but the L2 holds no "
-                    "dirty lines whose write-back the first reads would wait behind"}
-    return e
+    return {"workload": w.name, "ms_per_launch": ms, "tflops": tflops,
+            "frac_of_measured_peak": tflops / world / peak, "l2": l2_note}
 
 
 def our_arm(args, w):
@@ -548,18 +530,13 @@ def our_arm(args, w):
         del qd, kd, vd, od, kvd, flush_buf
         torch.cuda.empty_cache()
         configs = []
-        clean_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-        clean_buf.fill_(1)
         for cw in workloads.WORKLOADS:
             if cw.name == w.name:
                 configs.append(config_entry(cw, ms, world, peak, l2_note))
                 continue
-            cms, cnote, cclean = time_workload(torch, fa, cw, dev, stream, args.steps,
-                                               args.warmup, seed=cw.index + 1000 * rank,
-                                               clean_buf=clean_buf)
-            configs.append(config_entry(cw, max_over_ranks(cms, world), world, peak, cnote,
-                                        None if cclean is None else max_over_ranks(cclean, world)))
-        del clean_buf
+            cms, cnote = time_workload(torch, fa, cw, dev, stream, args.steps, args.warmup,
+                                       seed=cw.index + 1000 * rank)
+            configs.append(config_entry(cw, max_over_ranks(cms, world), world, peak, cnote))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -124,8 +124,8 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
 // tensor; box = 128 bytes of columns (the swizzle width) x box_rows rows x
 // box_planes heads. The third dimension keeps a tile from ever crossing into
 // the next head: rows past N read as zero.
-int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows = 128,
-             int box_planes = 1, int elem = 2) {
+int encode_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows,
+               int box_planes, int elem) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return FA_ERR_LAUNCH;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
@@ -138,6 +138,52 @@ int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_ro
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
+}
+
+// Encoded maps of recent calls, keyed by everything a map encodes (device,
+// address, shape, box, element size), so a loop that calls the library with
+// the same tensors pays for the encoding once. A map holds no reference to
+// the memory: a later tensor at the same address with the same shape gets the
+// same, still correct, map. Small and replaced round-robin.
+struct MapKey {
+    int dev;
+    const void* ptr;
+    int BH, N, d, box_rows, box_planes, elem;
+    bool operator==(const MapKey& o) const {
+        return dev == o.dev && ptr == o.ptr && BH == o.BH && N == o.N && d == o.d &&
+               box_rows == o.box_rows && box_planes == o.box_planes && elem == o.elem;
+    }
+};
+constexpr int kMapCache = 32;
+struct MapEntry {
+    bool used = false;
+    MapKey key{};
+    alignas(64) CUtensorMap map;
+};
+std::mutex g_map_mutex;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+
+int make_map(CUtensorMap* map, int dev, const void* ptr, int BH, int N, int d, int box_rows = 128,
+             int box_planes = 1, int elem = 2) {
+    const MapKey key{dev, ptr, BH, N, d, box_rows, box_planes, elem};
+    {
+        std::lock_guard<std::mutex> lk(g_map_mutex);
+        for (const MapEntry& e : g_maps)
+            if (e.used && e.key == key) {
+                *map = e.map;
+                return FA_OK;
+            }
+    }
+    const int rc = encode_map(map, ptr, BH, N, d, box_rows, box_planes, elem);
+    if (rc != FA_OK) return rc;
+    std::lock_guard<std::mutex> lk(g_map_mutex);
+    MapEntry& e = g_maps[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.used = true;
+    e.key = key;
+    e.map = *map;
+    return FA_OK;
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -186,8 +232,19 @@ void tile_shape(int H, int H_kv, int Nq, bool pack, int* G, int* nq_blk) {
     }
 }
 
-int fwd_impl(const FwdCall& a, void* stream) {
-    // ---- arguments (synchronous, nothing launched on error)
+// Shapes derived from a forward call's arguments.
+struct FwdPlan {
+    bool empty = false;      // B, H or Nq is 0: nothing to compute
+    int64_t BH = 0, BHkv = 0, BHB = 0, rows = 0, n_units = 0;
+    int G = 1, nq_blk = kTile, qt = 2;
+    bool general = false;
+    size_t tbytes = 0, lbytes = 0, qbytes = 0, kvbytes = 0;   // o, lse, q, k (= v) bytes
+};
+
+// Every host-side check of a forward call except its split-KV workspace
+// (synchronous, no CUDA call). Sizes are bounded before they are multiplied,
+// so no product can overflow.
+int fwd_check(const FwdCall& a, FwdPlan* pl) {
     const int B = a.B, H = a.H, H_kv = a.H_kv, Nq = a.Nq, Nk = a.Nk, d = a.d;
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || Nq > Nk) return FA_ERR_INVALID_ARG;
     if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_INVALID_ARG;
@@ -201,46 +258,63 @@ int fwd_impl(const FwdCall& a, void* stream) {
         for (float x : {a.q_descale, a.k_descale, a.v_descale})
             if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
     }
-    if (B == 0 || H == 0 || Nq == 0) return FA_OK;
+    if (B == 0 || H == 0 || Nq == 0) {
+        pl->empty = true;
+        return FA_OK;
+    }
     if (!a.q || !a.k || !a.v || !a.o || !a.lse) return FA_ERR_INVALID_ARG;
     const uintptr_t a16 = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
                           reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(a.o);
     if ((a16 & 15u) != 0 || (reinterpret_cast<uintptr_t>(a.lse) & 3u) != 0)
         return FA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(a.kv_len) & 3u) != 0) return FA_ERR_INVALID_ARG;
-    const int64_t BH = (int64_t)B * H;
-    const int64_t BHkv = (int64_t)B * H_kv;
-    int G = 1, nq_blk = kTile;
-    tile_shape(H, H_kv, Nq, a.pack, &G, &nq_blk);
+    // B, H, Nq < 2^31, so each product of two of them fits in int64
+    pl->BH = (int64_t)B * H;
+    pl->BHkv = (int64_t)B * H_kv;
+    if (pl->BH > INT32_MAX) return FA_ERR_INVALID_ARG;
+    pl->rows = pl->BH * Nq;
+    if (pl->rows > INT32_MAX) return FA_ERR_INVALID_ARG;   // row indices are 32-bit in the kernel
+    tile_shape(H, H_kv, Nq, a.pack, &pl->G, &pl->nq_blk);
     // Square attention (one key range, no packing, Nq == Nk) runs the
     // specialised kernels; everything else the general one-query-tile kernel.
-    const bool general = a.splits > 1 || G > 1 || Nq != Nk;
-    if (E == 1 && general) return FA_ERR_UNSUPPORTED;   // e4m3: square attention only
-    const int qt = (general || d == 256) ? 1 : 2;          // query tiles per unit
-    const int64_t n_rb = ((int64_t)Nq + nq_blk - 1) / nq_blk;
-    const int64_t n_units = (n_rb + qt - 1) / qt * a.splits;
-    const int64_t BHB = BH / G;
-    if (BH > INT32_MAX || BHB * n_units > INT32_MAX) return FA_ERR_INVALID_ARG;
-    if ((double)BH * Nq * d > 9.0e18 || (double)BHkv * Nk * d > 9.0e18) return FA_ERR_INVALID_ARG;
-    const int64_t rows = BH * Nq;
-    if (rows > INT32_MAX) return FA_ERR_INVALID_ARG;      // row indices are 32-bit in the kernel
-    const size_t tbytes = (size_t)rows * d * 2, lbytes = (size_t)rows * 4;
-    const size_t qbytes = (size_t)rows * d * E;
-    const size_t kvbytes = (size_t)BHkv * (size_t)Nk * (size_t)d * E;
-    if (overlaps(a.o, tbytes, a.q, qbytes) || overlaps(a.o, tbytes, a.k, kvbytes) ||
-        overlaps(a.o, tbytes, a.v, kvbytes) || overlaps(a.lse, lbytes, a.q, qbytes) ||
-        overlaps(a.lse, lbytes, a.k, kvbytes) || overlaps(a.lse, lbytes, a.v, kvbytes) ||
-        overlaps(a.lse, lbytes, a.o, tbytes))
+    pl->general = a.splits > 1 || pl->G > 1 || Nq != Nk;
+    if (E == 1 && pl->general) return FA_ERR_UNSUPPORTED;   // e4m3: square attention only
+    pl->qt = (pl->general || d == 256) ? 1 : 2;              // query tiles per unit
+    const int64_t n_rb = ((int64_t)Nq + pl->nq_blk - 1) / pl->nq_blk;
+    pl->n_units = (n_rb + pl->qt - 1) / pl->qt * a.splits;    // <= 2^31 * 128
+    pl->BHB = pl->BH / pl->G;
+    if (pl->n_units > INT32_MAX || pl->BHB > INT32_MAX / pl->n_units) return FA_ERR_INVALID_ARG;
+    if ((double)pl->BHkv * Nk * d > 9.0e18) return FA_ERR_INVALID_ARG;
+    pl->tbytes = (size_t)pl->rows * d * 2;
+    pl->lbytes = (size_t)pl->rows * 4;
+    pl->qbytes = (size_t)pl->rows * d * E;
+    pl->kvbytes = (size_t)pl->BHkv * (size_t)Nk * (size_t)d * E;
+    if (overlaps(a.o, pl->tbytes, a.q, pl->qbytes) || overlaps(a.o, pl->tbytes, a.k, pl->kvbytes) ||
+        overlaps(a.o, pl->tbytes, a.v, pl->kvbytes) ||
+        overlaps(a.lse, pl->lbytes, a.q, pl->qbytes) ||
+        overlaps(a.lse, pl->lbytes, a.k, pl->kvbytes) ||
+        overlaps(a.lse, pl->lbytes, a.v, pl->kvbytes) || overlaps(a.lse, pl->lbytes, a.o, pl->tbytes))
         return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+int fwd_impl(const FwdCall& a, void* stream) {
+    // ---- arguments (synchronous, nothing launched on error)
+    FwdPlan pl;
+    int rc = fwd_check(a, &pl);
+    if (rc != FA_OK || pl.empty) return rc;
+    const int B = a.B, H = a.H, H_kv = a.H_kv, Nq = a.Nq, Nk = a.Nk, d = a.d, E = a.elem;
+    const int64_t BH = pl.BH, BHkv = pl.BHkv, BHB = pl.BHB, rows = pl.rows, n_units = pl.n_units;
+    const int G = pl.G, nq_blk = pl.nq_blk;
     float* o_part = nullptr;
     float* lse_part = nullptr;
     if (a.splits > 1) {
         const size_t need = ws_total_bytes(rows, d, a.splits);
         if (a.ws == nullptr || a.ws_bytes < need || (reinterpret_cast<uintptr_t>(a.ws) & 15u) != 0)
             return FA_ERR_INVALID_ARG;
-        if (overlaps(a.ws, need, a.q, qbytes) || overlaps(a.ws, need, a.k, kvbytes) ||
-            overlaps(a.ws, need, a.v, kvbytes) || overlaps(a.ws, need, a.o, tbytes) ||
-            overlaps(a.ws, need, a.lse, lbytes))
+        if (overlaps(a.ws, need, a.q, pl.qbytes) || overlaps(a.ws, need, a.k, pl.kvbytes) ||
+            overlaps(a.ws, need, a.v, pl.kvbytes) || overlaps(a.ws, need, a.o, pl.tbytes) ||
+            overlaps(a.ws, need, a.lse, pl.lbytes))
             return FA_ERR_INVALID_ARG;
         o_part = static_cast<float*>(a.ws);
         lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
@@ -249,13 +323,13 @@ int fwd_impl(const FwdCall& a, void* stream) {
 
     int dev = 0;
     uint32_t* err = nullptr;
-    int rc = prepare_device(&dev, &err);
+    rc = prepare_device(&dev, &err);
     if (rc != FA_OK) return rc;
 
     alignas(64) CUtensorMap mq, mk, mv;
-    if ((rc = make_map(&mq, a.q, (int)BH, Nq, d, nq_blk, G, E)) != FA_OK) return rc;
-    if ((rc = make_map(&mk, a.k, (int)BHkv, Nk, d, 128, 1, E)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, a.v, (int)BHkv, Nk, d, 128, 1, E)) != FA_OK) return rc;
+    if ((rc = make_map(&mq, dev, a.q, (int)BH, Nq, d, nq_blk, G, E)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, dev, a.k, (int)BHkv, Nk, d, 128, 1, E)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, dev, a.v, (int)BHkv, Nk, d, 128, 1, E)) != FA_OK) return rc;
 
     FwdParams p{};
     p.o = static_cast<__nv_bfloat16*>(a.o);
@@ -272,7 +346,7 @@ int fwd_impl(const FwdCall& a, void* stream) {
     p.q_off = Nk - Nq;
     p.G = G;
     p.nq_blk = nq_blk;
-    p.n_rb = (int)n_rb;
+    p.n_rb = (int)(((int64_t)Nq + nq_blk - 1) / nq_blk);
     p.splits = a.splits;
     p.n_units = (int)n_units;
     // Launch-order head groups: as few groups as keep a group's K/V (2*Nk*d*2
@@ -296,7 +370,7 @@ int fwd_impl(const FwdCall& a, void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (E == 1) {
         fa_fwd_sm100<128, 2, false, 1><<<grid, block, Cfg<128, 2, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
-    } else if (general) {
+    } else if (pl.general) {
         if (d == 256)
             fa_fwd_sm100<256, 1, true><<<grid, block, Cfg<256, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
         else if (d == 128)
@@ -317,11 +391,14 @@ int fwd_impl(const FwdCall& a, void* stream) {
         const dim3 cblock(32 * kCombineWarps);
         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
         if (d == 256)
-            fa_splitkv_combine<256><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits);
+            fa_splitkv_combine<256><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits,
+                                                              err);
         else if (d == 128)
-            fa_splitkv_combine<128><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits);
+            fa_splitkv_combine<128><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits,
+                                                              err);
         else
-            fa_splitkv_combine<64><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits);
+            fa_splitkv_combine<64><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits,
+                                                              err);
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
     }
     return FA_OK;
@@ -379,9 +456,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     if ((a16 & 15u) != 0 || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
         (reinterpret_cast<uintptr_t>(kv_len) & 3u) != 0)
         return FA_ERR_INVALID_ARG;
-    const int64_t BH = (int64_t)B * H, BHkv = (int64_t)B * H_kv;
+    const int64_t BH = (int64_t)B * H, BHkv = (int64_t)B * H_kv;   // < 2^62
     const int64_t Np = bwd_np(N), n_t = Np / 128;
-    if (BH * Np > INT32_MAX || BH * n_t > INT32_MAX) return FA_ERR_INVALID_ARG;
+    if (BH > INT32_MAX || BH * Np > INT32_MAX) return FA_ERR_INVALID_ARG;
     if (ws_bytes < bwd_ws_bytes(BH, N)) return FA_ERR_INVALID_ARG;
     const size_t qb = (size_t)BH * N * d * 2, kb = (size_t)BHkv * N * d * 2;
     const size_t lb = (size_t)BH * N * 4, wb = bwd_ws_bytes(BH, N);
@@ -399,10 +476,10 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     int rc = prepare_device(&dev, &err);
     if (rc != FA_OK) return rc;
     alignas(64) CUtensorMap mq, mk, mv, mdo;
-    if ((rc = make_map(&mq, q, (int)BH, N, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mk, k, (int)BHkv, N, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, v, (int)BHkv, N, d)) != FA_OK) return rc;
-    if ((rc = make_map(&mdo, d_o, (int)BH, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mq, dev, q, (int)BH, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, dev, k, (int)BHkv, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, dev, v, (int)BHkv, N, d)) != FA_OK) return rc;
+    if ((rc = make_map(&mdo, dev, d_o, (int)BH, N, d)) != FA_OK) return rc;
 
     float* lse2 = static_cast<float*>(ws);
     float* dvec = lse2 + BH * Np;
@@ -480,9 +557,12 @@ FA_EXPORT int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, f
 }
 
 FA_EXPORT size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits) {
-    if (B < 0 || H < 0 || Nq < 0 || d < 0 || num_splits < 1 || num_splits > fa::kMaxSplits)
+    if (B < 0 || H < 0 || Nq < 0 || num_splits < 1 || num_splits > fa::kMaxSplits ||
+        (d != 64 && d != 128 && d != 256))
         return 0;
-    return fa::ws_total_bytes((int64_t)B * H * Nq, d, num_splits);
+    const int64_t bh = (int64_t)B * H;                  // < 2^62
+    if (bh > INT32_MAX || bh * Nq > INT32_MAX) return 0;
+    return fa::ws_total_bytes(bh * Nq, d, num_splits);
 }
 
 FA_EXPORT int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d) {
@@ -528,14 +608,15 @@ FA_EXPORT int fa_fwd_splitkv_static(const void* q, const void* k, const void* v,
     a.B = B; a.H = H; a.H_kv = H_kv; a.Nq = Nq; a.Nk = Nk; a.d = d;
     a.scale = scale; a.causal = causal; a.kv_len = kv_len;
     a.splits = num_splits; a.pack = true; a.ws = nullptr; a.ws_bytes = 0;
-    // Size check first, on the host: more partials than the scratch holds is
-    // an argument error, whatever else is wrong.
-    if (B > 0 && H > 0 && Nq > 0 && num_splits >= 1 && num_splits <= fa::kMaxSplits &&
-        fa::ws_total_bytes((int64_t)B * H * Nq, d, num_splits) > (size_t)FA_STATIC_SCRATCH_BYTES)
+    // The same argument checks as fa_fwd_splitkv, in the same order (so both
+    // entry points return the same status), then the scratch's size, all on
+    // the host before any CUDA call.
+    fa::FwdPlan pl;
+    const int arc = fa::fwd_check(a, &pl);
+    if (arc != FA_OK || pl.empty) return arc;
+    if (num_splits == 1) return fa::fwd_impl(a, stream);   // one range: no partials
+    if (fa::ws_total_bytes(pl.rows, d, num_splits) > (size_t)FA_STATIC_SCRATCH_BYTES)
         return FA_ERR_INVALID_ARG;
-    if (B <= 0 || H <= 0 || Nq <= 0 || num_splits < 2 || num_splits > fa::kMaxSplits ||
-        (d != 64 && d != 128 && d != 256))
-        return fa::fwd_impl(a, stream);   // empty problem, argument error or no partials
     void* scratch = nullptr;
     const int rc = fa::static_scratch(&scratch);
     if (rc != FA_OK) return rc;
@@ -557,7 +638,7 @@ FA_EXPORT int fa_fwd_fp8(const void* q, const void* k, const void* v, float q_de
 }
 
 FA_EXPORT size_t fa_bwd_workspace_bytes(int B, int H, int N) {
-    if (B < 0 || H < 0 || N < 0) return 0;
+    if (B < 0 || H < 0 || N < 0 || (int64_t)B * H > INT32_MAX) return 0;
     return fa::bwd_ws_bytes((int64_t)B * H, N);
 }
 

@@ -399,7 +399,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait_drain(&bars->teardown, 0u, wd);
         }
         __syncwarp();
-    } else if (!skip) {
+    } else if (skip) {
+        // An earlier kernel on this device timed out (the status word is
+        // sticky): no work, and this CTA's rows of dV (warpgroup 0) and dK
+        // (warpgroup 1) read NaN rather than stale memory.
+        const int jr = jt * 128 + (tid & 127);
+        if (jr < p.N)
+            fill_nan_bf16(((warp >> 2) != 0 ? p.dk : p.dv) + ((size_t)bkv * p.N + jr) * D, D);
+    } else {
         // ====================================================== compute warpgroups
         const int row = tid & 127;                     // TMEM lane = key row in the tile
         const int c0 = (warp >> 2) * 64;               // this warpgroup's half of the columns
@@ -614,7 +621,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait_drain(&bars->teardown, 0u, wd);
         }
         __syncwarp();
-    } else if (!skip) {
+    } else if (skip) {
+        // skipped launch (sticky status word): this CTA's half-rows of dQ read NaN
+        const int i = it * 128 + (tid & 127);
+        if (i < p.N)
+            fill_nan_bf16(p.dq + ((size_t)bh * p.N + i) * D + (warp >> 2) * (D / 2), D / 2);
+    } else {
         const int row = tid & 127;                     // TMEM lane = query row in the tile
         const int c0 = (warp >> 2) * 64;               // this warpgroup's half of the columns
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;

@@ -23,12 +23,23 @@ template <int D>
 __global__ void __launch_bounds__(32 * kCombineWarps)
     fa_splitkv_combine(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                        __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int64_t rows,
-                       int splits) {
+                       int splits, const uint32_t* dev_err) {
     constexpr int kPer = D / 32;   // columns per lane: 2, 4 or 8
     constexpr float kLog2e = 1.4426950408889634f;
     const int64_t row = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
+    if (*reinterpret_cast<const volatile uint32_t*>(dev_err) != 0u) {
+        // The attention kernel before this merge skipped or abandoned its work
+        // (the device status word is set): its partials are not this call's, so
+        // the row reads NaN instead of a merge of stale values.
+        const uint32_t nan2 = 0x7FC07FC0u;
+#pragma unroll
+        for (int c = 0; c < kPer; c += 2)
+            *reinterpret_cast<uint32_t*>(o + row * D + lane * kPer + c) = nan2;
+        if (lane == 0) lse[row] = __int_as_float(0x7FC00000);
+        return;
+    }
 
     // Pass 1: the largest lse_s (lane l reads splits l, l + 32, ...).
     float m = -INFINITY;

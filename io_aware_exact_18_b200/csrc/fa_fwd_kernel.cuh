@@ -246,6 +246,24 @@ __device__ __forceinline__ Unit decode_unit(int id, const FwdParams& p) {
     return u;
 }
 
+// Fill the O rows and lse entries of unit `id` with NaN (all threads of the
+// CTA take part): the output of a launch that skipped its work because the
+// device status word was already set.
+template <int D, int QT, bool kGen>
+__device__ void poison_unit(int id, const FwdParams& p, int tid, int nthreads) {
+    const Shape<kGen> sh(p);
+    const Unit u = decode_unit<QT, kGen>(id, p);
+    for (int e = tid; e < QT * kTile; e += nthreads) {
+        const int t = e / kTile, r = e - (e / kTile) * kTile;
+        const int g = r / sh.nq_blk;
+        const int i = (u.rb0 + t) * sh.nq_blk + (r - g * sh.nq_blk);
+        if (g >= sh.G || i >= sh.Nq) continue;
+        const size_t row = (size_t)(u.b * p.H + u.h0 + g) * sh.Nq + i;
+        fill_nan_bf16(p.o + row * D, D);
+        p.lse[row] = __int_as_float(0x7FC00000);
+    }
+}
+
 // Row maximum of a 128-score row held in registers.
 __device__ __forceinline__ float row_max(const float (&s)[kTile]) {
     float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
@@ -261,24 +279,61 @@ __device__ __forceinline__ float row_max(const float (&s)[kTile]) {
 
 // P = exp2(s*c - mc), rounded to bf16 pairs (E = 2: 64 TMEM columns) or to
 // e4m3 quadruples (E = 1: 32 columns) and written over the row's S in TMEM
-// (warp-wide stores); returns the row sum of the fp32 probabilities.
-template <int E>
-__device__ __forceinline__ float exp_tile(const float (&s)[kTile], float c, float mc,
-                                          uint32_t tS) {
+// (warp-wide stores). Returns two row sums: x, of the fp32 probabilities (the
+// exact sum, for lse and the overshoot test), and y, of the values as rounded
+// for the P.V product (bf16 P; for e4m3 P, y = x). O divided by y is a convex
+// combination of V rows whatever the rounding, so a row dominated by one key
+// returns that key's V row to within the output rounding, where O divided by x
+// would carry the dominant probability's rounding (up to 2^-8 of |V|): the
+// reference maximum of a row need not be its true maximum, so its largest
+// probability need not be exactly 1. kRounded = false skips the second sum
+// (y = x) for a caller that divides by the exact sum, and takes one scalar
+// instruction per score for the scale-subtract and the sum: the split-KV form
+// with two accumulators per row, whose packed pairs would spill registers.
+template <int E, bool kRounded = true>
+__device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, float mc,
+                                           uint32_t tS) {
     float sum0 = 0.f, sum1 = 0.f;
     if constexpr (E == 2) {
+        if constexpr (kRounded) {
+            float rs0 = 0.f, rs1 = 0.f;
+            float2 sum = make_float2(0.f, 0.f);
+            const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
 #pragma unroll
-        for (int ch = 0; ch < kTile / 32; ++ch) {
-            uint32_t packed[16];
+            for (int ch = 0; ch < kTile / 32; ++ch) {
+                uint32_t packed[16];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
-                const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
-                sum0 += p0;
-                sum1 += p1;
-                packed[q] = pack_bf16x2(p0, p1);
+                for (int q = 0; q < 16; ++q) {
+                    // The exponential pass is bound by instruction issue, not by
+                    // the MUFU pipe: the scale-subtract and the exact sum take one
+                    // packed (two-lane fp32) instruction per pair of scores.
+                    const float2 x = __ffma2_rn(
+                        make_float2(s[ch * 32 + 2 * q], s[ch * 32 + 2 * q + 1]), c2, nmc2);
+                    const float p0 = fast_exp2(x.x);
+                    const float p1 = fast_exp2(x.y);
+                    sum = __fadd2_rn(sum, make_float2(p0, p1));
+                    packed[q] = pack_bf16x2(p0, p1);
+                    rs0 = add_bf16_lo(packed[q], rs0);
+                    rs1 = add_bf16_hi(packed[q], rs1);
+                }
+                tmem_st16(tS + (uint32_t)(ch * 16), packed);
             }
-            tmem_st16(tS + (uint32_t)(ch * 16), packed);
+            return make_float2(sum.x + sum.y, rs0 + rs1);
+        } else {
+#pragma unroll
+            for (int ch = 0; ch < kTile / 32; ++ch) {
+                uint32_t packed[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
+                    const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
+                    sum0 += p0;
+                    sum1 += p1;
+                    packed[q] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tS + (uint32_t)(ch * 16), packed);
+            }
+            return make_float2(sum0 + sum1, sum0 + sum1);
         }
     } else {
 #pragma unroll
@@ -295,8 +350,8 @@ __device__ __forceinline__ float exp_tile(const float (&s)[kTile], float c, floa
             }
             tmem_st16(tS + (uint32_t)(ch * 16), packed);
         }
+        return make_float2(sum0 + sum1, sum0 + sum1);
     }
-    return sum0 + sum1;
 }
 
 // Largest row sum of a tile's probabilities before the row takes its true
@@ -371,6 +426,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem_base;
     const bool skip = bars->skip != 0;
     const Watchdog wd{&bars->abort, p.dev_err, p.watchdog_ns};
+    if (skip && (!kGen || p.o_part == nullptr)) {
+        // An earlier kernel on this device timed out (the status word is
+        // sticky): this launch does no attention work (the unit hand-out below
+        // publishes no unit, so every CTA of the grid runs just this) and each
+        // CTA fills its own unit's O and lse with NaN, so a caller who does not
+        // read the status word finds no stale values. Split-KV partials are
+        // left alone: the merge kernel checks the same word.
+        poison_unit<D, C::kQT, kGen>((int)blockIdx.x, p, tid, kThreads);
+    }
 
     if (warp == kTmaWarp) {
         // ====================================================== TMA producer + unit requests
@@ -718,6 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool idle_warp = kGen && !__any_sync(0xffffffffu, row_id >= 0);
             float m_ref = -INFINITY;   // reference maximum (raw score units)
             float l = 0.f;             // running sum of exp2((s - m_ref) * c)
+            float lr = 0.f;            // the same over the probabilities as rounded for P.V
             // tiles of this warpgroup: all of them, or (two accumulators) j = wg, wg + 2, ...
             const int j_first = kDual ? wg : 0, j_step = kDual ? 2 : 1;
             const int n_own = kDual ? (n > wg ? (n - wg + 1) / 2 : 0) : n;
@@ -782,20 +847,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float alpha = 1.f;
                 if (m_ref == -INFINITY) m_ref = row_max(s);
                 float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-                float l_tile = exp_tile<E>(s, c, mc, tS);
-                const bool stale = !(l_tile <= max_tile_sum<E>());
+                float2 l_tile = exp_tile<E, !kDual>(s, c, mc, tS);
+                const bool stale = !(l_tile.x <= max_tile_sum<E>());
                 if (__any_sync(0xffffffffu, stale)) {
                     if (stale) {
                         const float m_new = fmaxf(m_ref, row_max(s));
                         alpha = fast_exp2((m_ref - m_new) * c);
                         m_ref = m_new;
                         l *= alpha;
+                        lr *= alpha;
                         rescale = true;
                     }
                     mc = m_ref * c;
-                    l_tile = exp_tile<E>(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
+                    l_tile = exp_tile<E, !kDual>(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
                 }
-                l += l_tile;
+                l += l_tile.x;
+                lr += l_tile.y;
                 if (__any_sync(0xffffffffu, rescale)) {
                     // O holds the P.V sums of tiles < j: wait for the last of them,
                     // then bring it to the new reference maximum.
@@ -856,7 +923,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const bool write = row_id >= 0;
-            const float inv_l = (l > 0.f) ? p.o_mul / l : 0.f;
+            // O is divided by the sum of the rounded probabilities the P.V product
+            // used; lse takes the exact sum. (With two accumulators the merged
+            // divisor is the exact sum.)
+            const float o_div = kDual ? l : lr;
+            const float inv_l = (o_div > 0.f) ? p.o_mul / o_div : 0.f;
             const float row_lse = (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
             const size_t orow_idx = (size_t)row_id;
             const size_t prow_idx = (size_t)u.s * ((size_t)p.B * p.H * sh.Nq) + (size_t)row_id;

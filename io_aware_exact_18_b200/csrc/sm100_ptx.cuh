@@ -371,6 +371,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// acc + the low (element 0) or high (element 1) bf16 of a packed pair, the
+// bf16 widened exactly to fp32: one mixed-precision add, no unpacking.
+__device__ __forceinline__ float add_bf16_lo(uint32_t pk, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, lo, %2;\n\t}"
+        : "=f"(r) : "r"(pk), "f"(acc));
+    return r;
+}
+__device__ __forceinline__ float add_bf16_hi(uint32_t pk, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, hi, %2;\n\t}"
+        : "=f"(r) : "r"(pk), "f"(acc));
+    return r;
+}
+
+// Write n bf16 quiet NaNs (n a multiple of 8, dst 16-byte aligned): the
+// output of a launch that skipped its work because the device status word
+// was already set.
+__device__ __forceinline__ void fill_nan_bf16(__nv_bfloat16* dst, int n) {
+    const uint4 nan8 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int e = 0; e < n / 8; ++e) d4[e] = nan8;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -123,7 +123,10 @@ def test_bwd_is_deterministic(fa):
 
 def test_bwd_full_size_sampled(fa):
     """The backward the benchmark times (B1 H32 N16384 d128 causal, its inputs):
-    dQ on sampled rows of every head against the oracle's row-by-row dQ, and
+    dQ on sampled rows of every head against the oracle's row-by-row dQ; dK
+    and dV element by element on three key tiles (the first, which every
+    query row sees, one in the middle and the last, which few rows see) of
+    the first and the last head against the oracle's key-row gradients; and
     the two invariants of the definition for dK and dV on every head
     (sum_j dK_j = 0; sum_j dV_j = sum_i dO_i, every causal row seeing a key),
     each within 1 % of the summed magnitudes."""
@@ -136,6 +139,18 @@ def test_bwd_full_size_sampled(fa):
     err = np.abs(got - ref)
     assert err.max() <= MAX_REL * np.abs(ref).max() + ABS_FLOOR, f"dQ rows max|d| {err.max():.3e}"
     assert np.linalg.norm(err) <= FRO_REL * np.linalg.norm(ref) + ABS_FLOOR * math.sqrt(err.size)
+    heads = [0, w.H - 1]
+    keys = list(range(0, 128)) + list(range(w.N // 2, w.N // 2 + 128)) + \
+        list(range(w.N - 128, w.N))
+    sel = [x[:, heads].contiguous() for x in (q, k, v, do)]
+    dk_ref, dv_ref = oracle.attention_bwd_kv_rows(*sel, w.scale, keys, causal=True)
+    for name, g, r in (("dK", dk, dk_ref), ("dV", dv, dv_ref)):
+        got = g[:, heads][:, :, keys].double().cpu().numpy()
+        err = np.abs(got - r)
+        assert err.max() <= MAX_REL * np.abs(r).max() + ABS_FLOOR, \
+            f"{name} key rows max|d| {err.max():.3e} vs max|ref| {np.abs(r).max():.3e}"
+        assert np.linalg.norm(err) <= FRO_REL * np.linalg.norm(r) + \
+            ABS_FLOOR * math.sqrt(err.size), f"{name} key rows Frobenius error"
     dk64, dv64 = dk.double(), dv.double()
     sum_dk = dk64.sum(dim=2).abs().sum(dim=-1)
     assert torch.all(sum_dk <= 1e-2 * dk64.abs().sum(dim=(2, 3))), "sum_j dK_j != 0"

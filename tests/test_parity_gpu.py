@@ -76,29 +76,17 @@ def check_full(fa, q, k, v, causal, kv_len=None, scale=None, what=""):
 
 
 # ----------------------------------------------------------------- workloads
-@pytest.mark.parametrize("idx", [1, 2, 3])
+@pytest.mark.parametrize("idx", [1, 2, 3, 4, 5])
 def test_workload_full(fa, idx):
+    """Every element of every workload against the oracle, each at its full
+    size in the launch the benchmark times: the tiny case, BERT-large-shaped
+    key padding, GPT-2-shaped causal, the long-range case whose queries are
+    scaled by 4 (peaky rows that stress the running maximum and rescaling of
+    the online softmax) and the long-context case (about 2.2 TFLOP of fp64
+    oracle work, some 40 s on 16 host cores)."""
     w = workloads.get(idx)
     q, k, v, kv_len = workloads.make_inputs(w)
     check_full(fa, q, k, v, w.causal, kv_len, w.scale, w.name)
-
-
-@pytest.mark.parametrize("idx", [4, 5])
-def test_workload_sampled_rows(fa, idx):
-    """Full-size launch (the one the benchmark times); the oracle evaluates a
-    seeded sample of rows in every head: first/last 64 and 64 random."""
-    w = workloads.get(idx)
-    q, k, v, kv_len = workloads.make_inputs(w)
-    o, lse = run_gpu(fa, q, k, v, w.causal, kv_len, w.scale)
-    rows = workloads.sample_rows(w.N, seed=100 + idx, n_random=64, edge=64)
-    o_ref, lse_ref = oracle.attention(q, k, v, w.scale, causal=w.causal, kv_len=kv_len,
-                                      rows=rows)
-    compare(o[:, :, rows], lse[:, :, rows], o_ref, lse_ref, w.name)
-    # properties that hold at any size, on every row
-    assert np.isfinite(o).all() and np.isfinite(lse).all()
-    if w.causal:
-        v0 = v[:, :, 0].double().numpy()
-        assert np.abs(o[:, :, 0] - v0).max() <= 1e-2  # causal row 0 sees only key 0
 
 
 # ----------------------------------------------------------------- ragged / edge shapes
@@ -186,35 +174,79 @@ def test_grouped_heads_sampled_full_size(fa):
 
 
 def test_peaky_rows_rescale(fa):
-    """Large |scores| (Q x 8, far from the unit-normal scores the 2e-2 bound is
-    set for): rows are dominated by one or two keys, so the error is no longer
-    averaged over many weights. Its arithmetic bound: the bf16 rounding of each
-    probability (<= 2^-8 relative) moves O by at most 2^-8 * max|V|, and the
-    bf16 rounding of O adds at most 2^-8 * |O| <= 2^-8 * max|V|."""
+    """Large |scores| (Q x 8, far from unit-normal scores): rows are dominated by
+    one or two keys, whose weights the running reference maximum of the kernel
+    does not bring to exactly 1, so their bf16 rounding (up to 2^-8 relative)
+    would reach O if O were divided by the exact sum of the probabilities. The
+    kernel divides O by the sum of the probabilities as rounded for the P.V
+    product instead, which keeps such a row at its dominant V row to within the
+    output rounding, and the benchmark spec's bound holds: max |dO| <= 2e-2,
+    mean |dO| <= 2e-3, lse within 1e-3 (measured on a B200: 1.25e-2; 2.28e-2
+    with the exact sum as the divisor; 1.66e-2 for a kernel with an exact running
+    maximum)."""
     q, k, v, _ = workloads.make_custom(1, 4, 1024, 128, seed=9, q_mult=8.0)
-    bound = 2.0 ** -7 * float(v.float().abs().max())
     for causal in (False, True):
         o, lse = run_gpu(fa, q, k, v, causal, scale=1 / math.sqrt(128))
         o_ref, lse_ref = oracle.attention(q, k, v, 1 / math.sqrt(128), causal=causal)
-        err = np.abs(o - o_ref)
-        assert err.max() <= bound, f"Qx8 causal={causal}: max|dO| {err.max():.3e} > {bound:.3e}"
-        assert err.mean() <= MEAN_ABS
-        rel = np.abs(lse - lse_ref) / np.maximum(np.abs(lse_ref), 1.0)
-        assert rel.max() <= LSE_REL
+        err = compare(o, lse, o_ref, lse_ref, f"Qx8 causal={causal}")
+        print(f"Qx8 causal={causal}: max|dO| {err[0]:.4e} mean|dO| {err[1]:.4e}")
 
 
-def test_increasing_max_forces_rescale(fa):
-    """Scores that grow along the keys: every new tile raises the row max by
-    more than the rescale threshold, so every tile rescales O."""
-    N, d = 1024, 64
-    q = torch.zeros(1, 1, N, d)
-    q[..., 0] = 1.0
-    k = torch.zeros(1, 1, N, d)
-    k[0, 0, :, 0] = torch.linspace(0, 400, N)
-    v = torch.randn(1, 1, N, d, generator=torch.Generator().manual_seed(3))
+LOG2E = 1.4426950408889634
+
+
+def lazy_redo_counts(q, k, scale, causal, tile=128):
+    """Per query row, how many key tiles the kernel's reference-maximum rule
+    redoes: the row's first key tile sets the reference maximum m; a later
+    tile is exponentiated against m, and if its probabilities exp2((s - m) *
+    scale * log2 e) sum past 2^64 the row takes the tile's true maximum,
+    rescales O and l, and redoes the tile. Evaluated in fp64 from the bf16
+    inputs of one head."""
+    s = (q[0, 0].double() @ k[0, 0].double().T).numpy() * scale * LOG2E
+    n = s.shape[0]
+    counts = np.zeros(n, dtype=int)
+    for i in range(n):
+        row = s[i, :(i + 1 if causal else n)]
+        m = row[:tile].max()
+        for t0 in range(tile, row.shape[0], tile):
+            part = row[t0:t0 + tile]
+            if np.exp2(part - m).sum() > 2.0 ** 64:
+                m = max(m, part.max())
+                counts[i] += 1
+    return counts
+
+
+def test_redo_path_rescales_o(fa):
+    """Scores that climb tile by tile, so the reference-maximum rule redoes
+    tiles, at different rates within one warp. Query row i carries a_i in
+    {0, 1/8, 1/2, 1} (cycling, so every 32-row warp holds all four) in
+    column 0, key j carries 400 * (j // 128) there (exact in bf16), the other
+    columns small noise; with scale 1/8 a key tile raises a row's scores by
+    72 a_i in log2 units. Rows with a_i = 1 overshoot 2^64 on every tile and
+    redo seven; a_i = 1/2 every other tile; a_i = 1/8 once; a_i = 0 never
+    (lazy_redo_counts derives this from the rule). Without the redo, tile 7's
+    probabilities for a_i = 1 would be exp2(505) = inf in fp32 and O would not
+    be finite, so a finite O within the tolerance shows that the redo and the
+    O rescale ran."""
+    N, d, scale = 1024, 64, 0.125
+    g = torch.Generator().manual_seed(3)
+    q = 0.5 * torch.randn(1, 1, N, d, generator=g)
+    k = 0.5 * torch.randn(1, 1, N, d, generator=g)
+    v = torch.randn(1, 1, N, d, generator=g)
+    q[0, 0, :, 0] = torch.tensor([0.0, 0.125, 0.5, 1.0]).repeat(N // 4)
+    k[0, 0, :, 0] = 400.0 * (torch.arange(N) // 128).float()
     q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
-    check_full(fa, q, k, v, False, scale=0.125, what="monotone scores")
-    check_full(fa, q, k, v, True, scale=0.125, what="monotone scores causal")
+    assert torch.equal(k[0, 0, :, 0].float(), 400.0 * (torch.arange(N) // 128).float())
+    for causal in (False, True):
+        redos = lazy_redo_counts(q, k, scale, causal)
+        assert redos.max() == 7
+        first = 256 if causal else 0     # causal rows of the first two tiles see at most 2 tiles
+        for w0 in range(first, N, 32):   # every warp mixes rows that redo and rows that do not
+            warp = redos[w0:w0 + 32]
+            assert (warp >= 1).any() and (warp == 0).any(), (causal, w0, warp)
+        err = check_full(fa, q, k, v, causal, scale=scale, what=f"climbing scores causal={causal}")
+        print(f"climbing scores causal={causal}: redo tiles per row max {redos.max()}, "
+              f"total {redos.sum()}; max|dO| {err[0]:.3e} mean|dO| {err[1]:.3e}")
 
 
 # ----------------------------------------------------------------- pins on the GPU path
