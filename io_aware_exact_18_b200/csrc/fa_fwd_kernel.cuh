@@ -13,13 +13,16 @@
 // "Online softmax"). Exponentials use base 2 with the scale folded into one
 // FFMA per score, and the division by l is deferred to the epilogue, which
 // trims the non-matmul work that "FlashAttention-2 (HI)" section 1 targets.
-// The reference maximum m_ref is set by a row's first key tile and is only
-// raised when a later tile's probabilities, computed against it, would sum to
-// more than 2^64: each tile is exponentiated straight away, without first
-// reducing its row maximum, and the rare tile that overshoots is redone after
-// O and l are rescaled. Both O and l share the reference, so the final O / l
-// is unchanged by this choice (the ratio is exact), and every probability
-// stays below 2^64, far inside the fp32 and bf16 range.
+// The reference maximum m_ref is set by a row's first key tile and is raised
+// only rarely, so the per-tile rescale of the online softmax becomes an
+// exception. With two query tiles a tile's row maximum is taken before its
+// exponentials and moves m_ref only when it exceeds it by more than 64 in log2
+// units (8 for e4m3 P), after O and l are rescaled; with one query tile each
+// tile is exponentiated against m_ref straight away and the rare tile whose
+// probabilities would sum past 2^64 is redone after the rescale. Both O and l
+// share the reference, so the final O / l is unchanged by this choice (the
+// ratio is exact), and every probability stays at most 2^64, far inside the
+// fp32 and bf16 range.
 //
 // Work partitioning ("FlashAttention-2 (HI)", sections 2 and 3). A work unit
 // is one (batch, head, pair of 128-row query tiles) -- one tile at d = 256 --
@@ -94,7 +97,6 @@ constexpr int kTile = 128;         // rows per query tile and keys per KV tile
 constexpr int kThreads = 320;      // 2 softmax warpgroups + MMA warp + TMA warp
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
-constexpr float kMaxTileSum = 18446744073709551616.0f;  // 2^64
 constexpr float kLn2 = 0.69314718055994530942f;
 
 // Per head dimension and query tiles per unit. QT = 2 (square attention at
@@ -264,24 +266,28 @@ __device__ void poison_unit(int id, const FwdParams& p, int tid, int nthreads) {
     }
 }
 
-// Row maximum of a 128-score row held in registers.
+// Row maximum of a 128-score row held in registers: 64 three-input maxima in
+// four independent chains.
 __device__ __forceinline__ float row_max(const float (&s)[kTile]) {
+    static_assert(kTile == 128, "the chains below cover 128 scores");
     float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-    for (int q = 4; q < kTile; q += 4) {
-        mx0 = fmaxf(mx0, s[q]);
-        mx1 = fmaxf(mx1, s[q + 1]);
-        mx2 = fmaxf(mx2, s[q + 2]);
-        mx3 = fmaxf(mx3, s[q + 3]);
+    for (int q = 4; q < 116 + 8; q += 8) {
+        mx0 = fmax3(mx0, s[q], s[q + 1]);
+        mx1 = fmax3(mx1, s[q + 2], s[q + 3]);
+        mx2 = fmax3(mx2, s[q + 4], s[q + 5]);
+        mx3 = fmax3(mx3, s[q + 6], s[q + 7]);
     }
-    return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+    mx0 = fmax3(mx0, s[124], s[125]);
+    mx1 = fmax3(mx1, s[126], s[127]);
+    return fmaxf(fmax3(mx0, mx1, mx2), mx3);
 }
 
 // P = exp2(s*c - mc), rounded to bf16 pairs (E = 2: 64 TMEM columns) or to
-// e4m3 quadruples (E = 1: 32 columns) and written over the row's S in TMEM
-// (warp-wide stores). Returns two row sums: x, of the fp32 probabilities (the
-// exact sum, for lse and the overshoot test), and y, of the values as rounded
-// for the P.V product (bf16 P; for e4m3 P, y = x). O divided by y is a convex
+// e4m3 quadruples (E = 1: 32 columns) and written to TMEM at tP (warp-wide
+// stores, 16 columns at a time). Returns two row sums: x, of the fp32
+// probabilities (the exact sum, for lse), and y, of the values as rounded for
+// the P.V product (bf16 P; for e4m3 P, y = x). O divided by y is a convex
 // combination of V rows whatever the rounding, so a row dominated by one key
 // returns that key's V row to within the output rounding, where O divided by x
 // would carry the dominant probability's rounding (up to 2^-8 of |V|): the
@@ -292,7 +298,7 @@ __device__ __forceinline__ float row_max(const float (&s)[kTile]) {
 // with two accumulators per row, whose packed pairs would spill registers.
 template <int E, bool kRounded = true>
 __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, float mc,
-                                           uint32_t tS) {
+                                           uint32_t tP) {
     float sum0 = 0.f, sum1 = 0.f;
     if constexpr (E == 2) {
         if constexpr (kRounded) {
@@ -304,9 +310,8 @@ __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, flo
                 uint32_t packed[16];
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
-                    // The exponential pass is bound by instruction issue, not by
-                    // the MUFU pipe: the scale-subtract and the exact sum take one
-                    // packed (two-lane fp32) instruction per pair of scores.
+                    // The scale-subtract and the exact sum take one packed
+                    // (two-lane fp32) instruction per pair of scores.
                     const float2 x = __ffma2_rn(
                         make_float2(s[ch * 32 + 2 * q], s[ch * 32 + 2 * q + 1]), c2, nmc2);
                     const float p0 = fast_exp2(x.x);
@@ -316,7 +321,7 @@ __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, flo
                     rs0 = add_bf16_lo(packed[q], rs0);
                     rs1 = add_bf16_hi(packed[q], rs1);
                 }
-                tmem_st16(tS + (uint32_t)(ch * 16), packed);
+                tmem_st16(tP + (uint32_t)(ch * 16), packed);
             }
             return make_float2(sum.x + sum.y, rs0 + rs1);
         } else {
@@ -331,7 +336,7 @@ __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, flo
                     sum1 += p1;
                     packed[q] = pack_bf16x2(p0, p1);
                 }
-                tmem_st16(tS + (uint32_t)(ch * 16), packed);
+                tmem_st16(tP + (uint32_t)(ch * 16), packed);
             }
             return make_float2(sum0 + sum1, sum0 + sum1);
         }
@@ -348,18 +353,56 @@ __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, flo
                 sum1 += pq[1] + pq[3];
                 packed[q] = pack_e4m3x4(pq[0], pq[1], pq[2], pq[3]);
             }
-            tmem_st16(tS + (uint32_t)(ch * 16), packed);
+            tmem_st16(tP + (uint32_t)(ch * 16), packed);
         }
         return make_float2(sum0 + sum1, sum0 + sum1);
     }
 }
 
-// Largest row sum of a tile's probabilities before the row takes its true
-// maximum: 2^64 for bf16 P; 256 for e4m3 P, whose largest finite value is 448,
-// so every probability of an accepted tile is representable.
+// Two query tiles: a row's reference maximum is raised only when a tile's
+// maximum exceeds it by more than this (log2 units), so every probability is
+// at most 2^64 for bf16 P, or 2^8 for e4m3 P, whose largest finite value is 448.
 template <int E>
-__device__ __forceinline__ constexpr float max_tile_sum() {
-    return E == 2 ? kMaxTileSum : 256.0f;
+__device__ __forceinline__ constexpr float rescale_log2() {
+    return E == 2 ? 64.0f : 8.0f;
+}
+
+// One query tile: the largest row sum of a tile's probabilities, computed
+// against the reference, before the row takes its true maximum and the tile is
+// redone (2^64 for bf16 P).
+template <int E>
+__device__ __forceinline__ constexpr float redo_tile_sum() {
+    return E == 2 ? 18446744073709551616.0f : 256.0f;
+}
+
+// O (d columns of this thread's TMEM lane) *= alpha, kCols columns at a time.
+// With a tile's scores live (two query tiles) 16 columns in a rolled loop keep
+// the scores in registers; otherwise 32 columns fully unrolled (a rolled loop
+// there measured slower even though it rarely runs).
+template <int D, int kCols>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+    static_assert(kCols == 16 || kCols == 32, "TMEM load width");
+    if constexpr (kCols == 16) {
+#pragma unroll 1
+        for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t r[16];
+            tmem_ld16(tO + (uint32_t)(ch * 16), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
+            tmem_st16(tO + (uint32_t)(ch * 16), r);
+        }
+    } else {
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(tO + (uint32_t)(ch * 32), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
+            tmem_st32(tO + (uint32_t)(ch * 32), r);
+        }
+    }
 }
 
 template <int D, int QT, bool kGen, int E = 2>
@@ -376,6 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool kDual = kGen && QT == 1 && D <= 128;
     constexpr int kSoftmaxWarps = 4 * (kDual ? 2 : QT);
     constexpr int kConsumers = 1 + kSoftmaxWarps;   // MMA thread + one lane per softmax warp
+    // Reference-maximum rule (see the softmax loop): fixed before the
+    // exponentials with two query tiles, where it measured faster; exponentiate
+    // first and redo the rare overshooting tile with one (S double-buffered, the
+    // row maximum pass would sit on the critical path).
+    constexpr bool kMaxFirst = QT == 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -495,15 +543,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bars->unit_full[us]);
                 if (id < 0) break;
                 const Unit u = decode_unit<C::kQT, kGen>(id, p);
-                // The first two K/V loads go first: the ring has room while the
-                // previous unit's last tiles are consumed, and Q may have to wait.
-                const int early = min(2, 2 * u.n_max);
-                for (int jj = 0; ok && jj < early; ++jj) ok = load_kv(u, jj);
-                // Q tiles (one q_full phase per unit and tile, possibly with no
+                // Q tile t (one q_full phase per unit and tile, possibly with no
                 // bytes). One box per 64-column block: nq_blk rows of G heads.
-                for (int t = 0; t < C::kQT && ok; ++t) {
-                    if (k > 0) ok = mbar_wait(&bars->q_empty[t], (uint32_t)((k - 1) & 1), wd);
-                    if (!ok) break;
+                auto load_q = [&](int t) -> bool {
+                    if (k > 0 && !mbar_wait(&bars->q_empty[t], (uint32_t)((k - 1) & 1), wd))
+                        return false;
                     mbar_arrive_expect_tx(&bars->q_full[t], u.n[t] > 0 ? q_bytes : 0u);
                     q_unit[t] = k;
                     if (u.n[t] > 0)
@@ -511,7 +555,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_3d_hint(&tm_q, &bars->q_full[t], sQ[t] + blk * C::kBlockBytes,
                                              blk * C::kBlockElems, (u.rb0 + t) * sh.nq_blk,
                                              u.b * p.H + u.h0, pol_q);
-                }
+                    return true;
+                };
+                // The first two K/V loads go first: the ring has room while the
+                // previous unit's last tiles are consumed, and Q may have to wait.
+                const int early = min(2, 2 * u.n_max);
+                for (int jj = 0; ok && jj < early; ++jj) ok = load_kv(u, jj);
+                for (int t = 0; ok && t < C::kQT; ++t) ok = load_q(t);
                 // the rest of K_0, V_0, K_1, V_1, ... of this unit
                 for (int jj = early; ok && jj < 2 * u.n_max; ++jj) ok = load_kv(u, jj);
                 if (!ok) break;
@@ -574,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // blocks (the same instruction shape as d = 128).
             auto issue_pv = [&](int t, int sb, int slot, bool accumulate) {
                 const uint64_t b = dv0 + (uint64_t)slot * kTileStep;
+                const uint32_t tP = tmem + C::col_s(sb);
 #pragma unroll
                 for (int kk = 0; kk < kTile / kStepRows; ++kk) {
 #pragma unroll
@@ -582,10 +633,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                             h * (kPvN / 64) * C::kBlockBytes) >> 4);
                         if constexpr (E == 2)
                             umma_ts(tmem + C::col_o(t) + (uint32_t)(h * kPvN),
-                                    tmem + C::col_s(sb) + (uint32_t)(kk * 8), bk, idesc_pv,
+                                    tP + (uint32_t)(kk * 8), bk, idesc_pv,
                                     (accumulate || kk > 0) ? 1u : 0u);
                         else
-                            umma_ts_f8(tmem + C::col_o(t), tmem + C::col_s(sb) + (uint32_t)(kk * 8),
+                            umma_ts_f8(tmem + C::col_o(t), tP + (uint32_t)(kk * 8),
                                        bk, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
                     }
                 }
@@ -836,49 +887,77 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int q = 0; q < kTile; ++q)
                         if (q >= lim) s[q] = -INFINITY;
                 }
-                // The first tile sets the reference maximum m_ref from its row
-                // maximum. Later tiles exponentiate against the current m_ref
-                // straight away; only if that makes the tile's row sum exceed
-                // 2^64 (some p > 2^64) does the row take its true maximum,
-                // rescale O and l, and redo the tile. Below that bound every
-                // probability, l (< N * 2^64) and O stay far inside the fp32
-                // and bf16 range, and O / l is exact whatever m_ref is.
                 bool rescale = false;
                 float alpha = 1.f;
-                if (m_ref == -INFINITY) m_ref = row_max(s);
-                float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-                float2 l_tile = exp_tile<E, !kDual>(s, c, mc, tS);
-                const bool stale = !(l_tile.x <= max_tile_sum<E>());
-                if (__any_sync(0xffffffffu, stale)) {
-                    if (stale) {
-                        const float m_new = fmaxf(m_ref, row_max(s));
-                        alpha = fast_exp2((m_ref - m_new) * c);
-                        m_ref = m_new;
+                float2 l_tile;
+                if constexpr (kMaxFirst) {
+                    // The reference maximum m_ref is fixed before any exponential
+                    // of the tile: the row's first visible tile sets it to its row
+                    // maximum, and a later tile moves it only when the tile's
+                    // maximum exceeds it by more than rescale_log2 (log2 units),
+                    // after O and l are brought to the new reference. Every
+                    // probability is then at most 2^64 (bf16 P), l < N * 2^64 and
+                    // O stay far inside the fp32 range, and O / l is exact
+                    // whatever m_ref is.
+                    const float m_tile = row_max(s);
+                    if (m_ref == -INFINITY) {
+                        m_ref = m_tile;
+                    } else if ((m_tile - m_ref) * c > rescale_log2<E>()) {
+                        alpha = fast_exp2((m_ref - m_tile) * c);
+                        m_ref = m_tile;
                         l *= alpha;
                         lr *= alpha;
                         rescale = true;
                     }
-                    mc = m_ref * c;
-                    l_tile = exp_tile<E, !kDual>(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
-                }
-                l += l_tile.x;
-                lr += l_tile.y;
-                if (__any_sync(0xffffffffu, rescale)) {
-                    // O holds the P.V sums of tiles < j: wait for the last of them,
-                    // then bring it to the new reference maximum.
-                    ok = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(jo - 1)) & 1u, wd);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch) {
-                        uint32_t r[32];
-                        tmem_ld32(tO + (uint32_t)(ch * 32), r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 32; ++q)
-                            r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
-                        tmem_st32(tO + (uint32_t)(ch * 32), r);
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        // O holds the P.V sums of tiles < j: wait for the last of
+                        // them (P of this tile is not handed over yet, so o_done is
+                        // exactly at that phase or one short), then rescale it, 16
+                        // columns at a time while the tile's scores are live.
+                        ok = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(jo - 1)) & 1u, wd);
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        tc_fence_after();
+                        rescale_o<D, 16>(tO, alpha);
+                    }
+                    const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+                    l_tile = exp_tile<E, !kDual>(s, c, mc, tS);
+                    l += l_tile.x;
+                    lr += l_tile.y;
+                } else {
+                    // The first tile sets the reference maximum m_ref from its row
+                    // maximum. Later tiles exponentiate against the current m_ref
+                    // straight away; only if that makes the tile's row sum exceed
+                    // redo_tile_sum (some p > 2^64) does the row take its true
+                    // maximum, rescale O and l, and redo the tile. Below that bound
+                    // every probability, l (< N * 2^64) and O stay far inside the
+                    // fp32 and bf16 range, and O / l is exact whatever m_ref is.
+                    if (m_ref == -INFINITY) m_ref = row_max(s);
+                    float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+                    l_tile = exp_tile<E, !kDual>(s, c, mc, tS);
+                    const bool stale = !(l_tile.x <= redo_tile_sum<E>());
+                    if (__any_sync(0xffffffffu, stale)) {
+                        if (stale) {
+                            const float m_new = fmaxf(m_ref, row_max(s));
+                            alpha = fast_exp2((m_ref - m_new) * c);
+                            m_ref = m_new;
+                            l *= alpha;
+                            lr *= alpha;
+                            rescale = true;
+                        }
+                        mc = m_ref * c;
+                        l_tile = exp_tile<E, !kDual>(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
+                    }
+                    l += l_tile.x;
+                    lr += l_tile.y;
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        // O holds the P.V sums of tiles < j: wait for the last of
+                        // them, then bring it to the new reference maximum.
+                        ok = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(jo - 1)) & 1u, wd);
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        tc_fence_after();
+                        rescale_o<D, 32>(tO, alpha);
                     }
                 }
                 tmem_wait_st();
@@ -931,23 +1010,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float row_lse = (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
             const size_t orow_idx = (size_t)row_id;
             const size_t prow_idx = (size_t)u.s * ((size_t)p.B * p.H * sh.Nq) + (size_t)row_id;
+            // O leaves TMEM kW columns at a time (16 with two accumulators,
+            // whose columns are both live at once).
+            constexpr int kW = kDual ? 16 : 32;
+            auto ld_cols = [&](uint32_t taddr, uint32_t (&r)[kW]) {
+                if constexpr (kW == 16) tmem_ld16(taddr, r);
+                else tmem_ld32(taddr, r);
+            };
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t r[32];
+            for (int ch = 0; ch < D / kW; ++ch) {
+                uint32_t r[kW];
                 if (n > 0 && !idle_warp) {
-                    tmem_ld32(tO + (uint32_t)(ch * 32), r);
+                    ld_cols(tO + (uint32_t)(ch * kW), r);
                     if constexpr (kDual) {
-                        uint32_t r1[32];
+                        uint32_t r1[kW];
                         if (have1) {
-                            tmem_ld32(tmem + lane_base + C::col_o(1) + (uint32_t)(ch * 32), r1);
+                            ld_cols(tmem + lane_base + C::col_o(1) + (uint32_t)(ch * kW), r1);
                             tmem_wait_ld();
                         } else {
                             tmem_wait_ld();
 #pragma unroll
-                            for (int q = 0; q < 32; ++q) r1[q] = 0u;
+                            for (int q = 0; q < kW; ++q) r1[q] = 0u;
                         }
 #pragma unroll
-                        for (int q = 0; q < 32; ++q)
+                        for (int q = 0; q < kW; ++q)
                             r[q] = __float_as_uint(__uint_as_float(r[q]) * a0 +
                                                    __uint_as_float(r1[q]) * a1);
                     } else {
@@ -955,18 +1041,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) r[q] = 0u;
+                    for (int q = 0; q < kW; ++q) r[q] = 0u;
                 }
-                if (ch == D / 32 - 1) {
+                if (ch == D / kW - 1) {
                     // O has been read: the next unit's first P.V may overwrite it
                     tc_fence_before();
                     mbar_arrive(&bars->o_empty[ob]);
                     if (kDual) mbar_arrive(&bars->o_empty[1]);
                 }
                 if (write && (!kGen || p.o_part == nullptr)) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow_idx * D + ch * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow_idx * D + ch * kW);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
+                    for (int v = 0; v < kW / 8; ++v) {
                         uint4 w;
                         w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv_l,
                                           __uint_as_float(r[8 * v + 1]) * inv_l);
@@ -980,9 +1066,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 } else if (write) {
                     // split-KV partial: this key range's O / l in fp32
-                    float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * D + ch * 32);
+                    float4* dst = reinterpret_cast<float4*>(p.o_part + prow_idx * D + ch * kW);
 #pragma unroll
-                    for (int v = 0; v < 8; ++v)
+                    for (int v = 0; v < kW / 4; ++v)
                         dst[v] = make_float4(__uint_as_float(r[4 * v + 0]) * inv_l,
                                              __uint_as_float(r[4 * v + 1]) * inv_l,
                                              __uint_as_float(r[4 * v + 2]) * inv_l,

@@ -195,13 +195,13 @@ def test_peaky_rows_rescale(fa):
 LOG2E = 1.4426950408889634
 
 
-def lazy_redo_counts(q, k, scale, causal, tile=128):
-    """Per query row, how many key tiles the kernel's reference-maximum rule
-    redoes: the row's first key tile sets the reference maximum m; a later
-    tile is exponentiated against m, and if its probabilities exp2((s - m) *
-    scale * log2 e) sum past 2^64 the row takes the tile's true maximum,
-    rescales O and l, and redoes the tile. Evaluated in fp64 from the bf16
-    inputs of one head."""
+def reference_moves(q, k, scale, causal, tile=128):
+    """Per query row, how many key tiles move the kernel's reference maximum:
+    the row's first key tile sets the reference m to its maximum; a later
+    tile whose maximum exceeds m by more than 64 in log2 units (some
+    probability exp2((s - m) * scale * log2 e) would pass 2^64) makes the row
+    take that maximum, rescaling O and l before the tile is exponentiated.
+    Evaluated in fp64 from the bf16 inputs of one head."""
     s = (q[0, 0].double() @ k[0, 0].double().T).numpy() * scale * LOG2E
     n = s.shape[0]
     counts = np.zeros(n, dtype=int)
@@ -210,24 +210,24 @@ def lazy_redo_counts(q, k, scale, causal, tile=128):
         m = row[:tile].max()
         for t0 in range(tile, row.shape[0], tile):
             part = row[t0:t0 + tile]
-            if np.exp2(part - m).sum() > 2.0 ** 64:
-                m = max(m, part.max())
+            if part.max() - m > 64.0:
+                m = part.max()
                 counts[i] += 1
     return counts
 
 
-def test_redo_path_rescales_o(fa):
-    """Scores that climb tile by tile, so the reference-maximum rule redoes
-    tiles, at different rates within one warp. Query row i carries a_i in
+def test_reference_move_rescales_o(fa):
+    """Scores that climb tile by tile, so the reference maximum moves, at
+    different rates within one warp. Query row i carries a_i in
     {0, 1/8, 1/2, 1} (cycling, so every 32-row warp holds all four) in
     column 0, key j carries 400 * (j // 128) there (exact in bf16), the other
     columns small noise; with scale 1/8 a key tile raises a row's scores by
-    72 a_i in log2 units. Rows with a_i = 1 overshoot 2^64 on every tile and
-    redo seven; a_i = 1/2 every other tile; a_i = 1/8 once; a_i = 0 never
-    (lazy_redo_counts derives this from the rule). Without the redo, tile 7's
-    probabilities for a_i = 1 would be exp2(505) = inf in fp32 and O would not
-    be finite, so a finite O within the tolerance shows that the redo and the
-    O rescale ran."""
+    72 a_i in log2 units. Rows with a_i = 1 move their reference maximum on
+    every later tile (seven times); a_i = 1/2 every other tile; a_i = 1/8 at
+    most once; a_i = 0 never (reference_moves derives this from the rule).
+    Without the move, tile 7's probabilities for a_i = 1 would be exp2(505) =
+    inf in fp32 and O would not be finite, so a finite O within the tolerance
+    shows that the rescale of O and l ran."""
     N, d, scale = 1024, 64, 0.125
     g = torch.Generator().manual_seed(3)
     q = 0.5 * torch.randn(1, 1, N, d, generator=g)
@@ -238,15 +238,15 @@ def test_redo_path_rescales_o(fa):
     q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
     assert torch.equal(k[0, 0, :, 0].float(), 400.0 * (torch.arange(N) // 128).float())
     for causal in (False, True):
-        redos = lazy_redo_counts(q, k, scale, causal)
-        assert redos.max() == 7
+        moves = reference_moves(q, k, scale, causal)
+        assert moves.max() == 7
         first = 256 if causal else 0     # causal rows of the first two tiles see at most 2 tiles
-        for w0 in range(first, N, 32):   # every warp mixes rows that redo and rows that do not
-            warp = redos[w0:w0 + 32]
+        for w0 in range(first, N, 32):   # every warp mixes rows that move their reference and rows that do not
+            warp = moves[w0:w0 + 32]
             assert (warp >= 1).any() and (warp == 0).any(), (causal, w0, warp)
         err = check_full(fa, q, k, v, causal, scale=scale, what=f"climbing scores causal={causal}")
-        print(f"climbing scores causal={causal}: redo tiles per row max {redos.max()}, "
-              f"total {redos.sum()}; max|dO| {err[0]:.3e} mean|dO| {err[1]:.3e}")
+        print(f"climbing scores causal={causal}: reference moves per row max {moves.max()}, "
+              f"total {moves.sum()}; max|dO| {err[0]:.3e} mean|dO| {err[1]:.3e}")
 
 
 # ----------------------------------------------------------------- pins on the GPU path
