@@ -196,12 +196,13 @@ LOG2E = 1.4426950408889634
 
 
 def reference_moves(q, k, scale, causal, tile=128):
-    """Per query row, how many key tiles move the kernel's reference maximum:
-    the row's first key tile sets the reference m to its maximum; a later
-    tile whose maximum exceeds m by more than 64 in log2 units (some
-    probability exp2((s - m) * scale * log2 e) would pass 2^64) makes the row
-    take that maximum, rescaling O and l before the tile is exponentiated.
-    Evaluated in fp64 from the bf16 inputs of one head."""
+    """Per query row, how many key tiles move the reference maximum of the
+    two-query-tile kernel (d <= 128): the row's first key tile sets the
+    reference m to its maximum; a later tile whose maximum exceeds m by more
+    than 64 in log2 units (some probability exp2((s - m) * scale * log2 e)
+    would pass 2^64) makes the row take that maximum, rescaling O and l before
+    the tile is exponentiated. Evaluated in fp64 from the bf16 inputs of one
+    head."""
     s = (q[0, 0].double() @ k[0, 0].double().T).numpy() * scale * LOG2E
     n = s.shape[0]
     counts = np.zeros(n, dtype=int)
@@ -216,7 +217,28 @@ def reference_moves(q, k, scale, causal, tile=128):
     return counts
 
 
-def test_reference_move_rescales_o(fa):
+def reference_redos(q, k, scale, causal, tile=128):
+    """The same count for the one-query-tile kernel (d = 256): the first key
+    tile sets m to its maximum; a later tile is exponentiated against m and,
+    if its probabilities exp2((s - m) * scale * log2 e) sum past 2^64, the row
+    takes the larger of m and the tile's maximum, rescales O and l, and redoes
+    the tile."""
+    s = (q[0, 0].double() @ k[0, 0].double().T).numpy() * scale * LOG2E
+    n = s.shape[0]
+    counts = np.zeros(n, dtype=int)
+    for i in range(n):
+        row = s[i, :(i + 1 if causal else n)]
+        m = row[:tile].max()
+        for t0 in range(tile, row.shape[0], tile):
+            part = row[t0:t0 + tile]
+            if np.exp2(part - m).sum() > 2.0 ** 64:
+                m = max(m, part.max())
+                counts[i] += 1
+    return counts
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_reference_move_rescales_o(fa, d):
     """Scores that climb tile by tile, so the reference maximum moves, at
     different rates within one warp. Query row i carries a_i in
     {0, 1/8, 1/2, 1} (cycling, so every 32-row warp holds all four) in
@@ -224,28 +246,31 @@ def test_reference_move_rescales_o(fa):
     columns small noise; with scale 1/8 a key tile raises a row's scores by
     72 a_i in log2 units. Rows with a_i = 1 move their reference maximum on
     every later tile (seven times); a_i = 1/2 every other tile; a_i = 1/8 at
-    most once; a_i = 0 never (reference_moves derives this from the rule).
-    Without the move, tile 7's probabilities for a_i = 1 would be exp2(505) =
-    inf in fp32 and O would not be finite, so a finite O within the tolerance
-    shows that the rescale of O and l ran."""
-    N, d, scale = 1024, 64, 0.125
+    most once; a_i = 0 never. d = 64 runs the two-tile kernel (maximum taken
+    before the exponentials, reference_moves), d = 256 the one-tile kernel
+    (exponentiate, redo past 2^64, reference_redos). Without the move, tile
+    7's probabilities for a_i = 1 would be exp2(505) = inf in fp32 and O would
+    not be finite, so a finite O within the tolerance shows that the rescale
+    of O and l ran."""
+    N, scale = 1024, 0.125
     g = torch.Generator().manual_seed(3)
-    q = 0.5 * torch.randn(1, 1, N, d, generator=g)
+    q = 0.5 * torch.randn(1, 1, N, d, generator=g) * (64 / d) ** 0.5
     k = 0.5 * torch.randn(1, 1, N, d, generator=g)
     v = torch.randn(1, 1, N, d, generator=g)
     q[0, 0, :, 0] = torch.tensor([0.0, 0.125, 0.5, 1.0]).repeat(N // 4)
     k[0, 0, :, 0] = 400.0 * (torch.arange(N) // 128).float()
     q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
     assert torch.equal(k[0, 0, :, 0].float(), 400.0 * (torch.arange(N) // 128).float())
+    rule = reference_moves if d <= 128 else reference_redos
     for causal in (False, True):
-        moves = reference_moves(q, k, scale, causal)
+        moves = rule(q, k, scale, causal)
         assert moves.max() == 7
         first = 256 if causal else 0     # causal rows of the first two tiles see at most 2 tiles
         for w0 in range(first, N, 32):   # every warp mixes rows that move their reference and rows that do not
             warp = moves[w0:w0 + 32]
             assert (warp >= 1).any() and (warp == 0).any(), (causal, w0, warp)
-        err = check_full(fa, q, k, v, causal, scale=scale, what=f"climbing scores causal={causal}")
-        print(f"climbing scores causal={causal}: reference moves per row max {moves.max()}, "
+        err = check_full(fa, q, k, v, causal, scale=scale, what=f"climbing scores causal={causal} d={d}")
+        print(f"climbing scores causal={causal} d={d}: reference moves per row max {moves.max()}, "
               f"total {moves.sum()}; max|dO| {err[0]:.3e} mean|dO| {err[1]:.3e}")
 
 
