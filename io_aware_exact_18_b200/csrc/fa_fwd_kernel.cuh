@@ -121,7 +121,7 @@ struct Cfg {
     static constexpr int kSlots =                         // K/V ring depth
         (E == 1) ? 8 : (D == 256) ? 2 : (D == 128) ? (QT == 2 ? 4 : 5) : 8;
     static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
-    static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 3072 /*barriers*/;
+    static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 4096 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
     // S buffer b (a query tile's, or with one tile the buffer of key-tile parity b)
     __device__ static constexpr uint32_t col_s(int b) { return (uint32_t)(b * 128); }
@@ -169,14 +169,15 @@ struct SmemBarriers {
     uint64_t kv_empty[8];
     uint64_t merge_full[2];    // two-accumulator mode: warpgroup 1's (m, l) per row, by unit parity
     float merge_m[2][kTile];
-    float merge_l[2][kTile];
+    float merge_l[2][kTile];   // exact row sum
+    float merge_lr[2][kTile];  // sum of the rounded probabilities
     uint4 clc_resp[2];         // 16-byte aligned (offset is a multiple of 16)
     int unit_id[2];
     uint32_t tmem_base;
     int abort;
     int skip;
 };
-static_assert(sizeof(SmemBarriers) <= 3072, "barrier region");
+static_assert(sizeof(SmemBarriers) <= 4096, "barrier region");
 static_assert(offsetof(SmemBarriers, clc_resp) % 16 == 0, "CLC response alignment");
 
 // One work unit, decoded from its launch-order index. A tile's 128 rows hold
@@ -292,16 +293,16 @@ __device__ __forceinline__ float row_max(const float (&s)[kTile]) {
 // returns that key's V row to within the output rounding, where O divided by x
 // would carry the dominant probability's rounding (up to 2^-8 of |V|): the
 // reference maximum of a row need not be its true maximum, so its largest
-// probability need not be exactly 1. kRounded = false skips the second sum
-// (y = x) for a caller that divides by the exact sum, and takes one scalar
-// instruction per score for the scale-subtract and the sum: the split-KV form
-// with two accumulators per row, whose packed pairs would spill registers.
-template <int E, bool kRounded = true>
+// probability need not be exactly 1. kPacked = false takes one scalar
+// instruction per score for the scale-subtract and the exact sum instead of
+// one packed (two-lane) instruction per pair: the split-KV form with two
+// accumulators per row, whose packed pairs would spill registers.
+template <int E, bool kPacked = true>
 __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, float mc,
                                            uint32_t tP) {
     float sum0 = 0.f, sum1 = 0.f;
     if constexpr (E == 2) {
-        if constexpr (kRounded) {
+        if constexpr (kPacked) {
             float rs0 = 0.f, rs1 = 0.f;
             float2 sum = make_float2(0.f, 0.f);
             const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
@@ -325,6 +326,7 @@ __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, flo
             }
             return make_float2(sum.x + sum.y, rs0 + rs1);
         } else {
+            float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
             for (int ch = 0; ch < kTile / 32; ++ch) {
                 uint32_t packed[16];
@@ -335,10 +337,12 @@ __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, flo
                     sum0 += p0;
                     sum1 += p1;
                     packed[q] = pack_bf16x2(p0, p1);
+                    rs0 = add_bf16_lo(packed[q], rs0);
+                    rs1 = add_bf16_hi(packed[q], rs1);
                 }
                 tmem_st16(tP + (uint32_t)(ch * 16), packed);
             }
-            return make_float2(sum0 + sum1, sum0 + sum1);
+            return make_float2(sum0 + sum1, rs0 + rs1);
         }
     } else {
 #pragma unroll
@@ -975,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(&bars->o_done[ob], last & 1u, wd);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            // Two accumulators: warpgroup 1 hands its row's (m, l) to warpgroup 0
+            // Two accumulators: warpgroup 1 hands its row's (m, l, lr) to warpgroup 0
             // (its O1 is complete: it has just waited for its last P.V), and
             // warpgroup 0 writes the merged row.
             float a0 = 1.f, a1 = 0.f;          // weights of O0 and O1 in the merged row
@@ -985,6 +989,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (wg == 1) {
                     bars->merge_m[mb][row] = (l > 0.f) ? m_ref * c : -INFINITY;
                     bars->merge_l[mb][row] = l;
+                    bars->merge_lr[mb][row] = lr;
                     mbar_arrive(&bars->merge_full[mb]);
                     continue;
                 }
@@ -997,15 +1002,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a0 = (l > 0.f) ? fast_exp2(m0 - mm) : 0.f;
                 a1 = (l1 > 0.f) ? fast_exp2(m1 - mm) : 0.f;
                 l = l * a0 + l1 * a1;
+                lr = lr * a0 + bars->merge_lr[mb][row] * a1;
                 m_ref = (mm == -INFINITY) ? -INFINITY : mm / c;   // merged reference (score units)
                 have1 = n > 1;
             }
             tc_fence_after();
             const bool write = row_id >= 0;
             // O is divided by the sum of the rounded probabilities the P.V product
-            // used; lse takes the exact sum. (With two accumulators the merged
-            // divisor is the exact sum.)
-            const float o_div = kDual ? l : lr;
+            // used (with two accumulators, both sums merged like O); lse takes
+            // the exact sum.
+            const float o_div = lr;
             const float inv_l = (o_div > 0.f) ? p.o_mul / o_div : 0.f;
             const float row_lse = (l > 0.f) ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
             const size_t orow_idx = (size_t)row_id;
