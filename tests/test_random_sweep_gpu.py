@@ -83,3 +83,53 @@ def test_random_configuration(fa, case):
             f"q x {q_mult} splits={splits}")
     err = compare(out.double().cpu().numpy(), lse.double().cpu().numpy(), o_ref, lse_ref, what)
     print(f"{what}: max|dO| {err[0]:.2e} mean|dO| {err[1]:.2e}")
+
+
+N_BWD_CASES = 24
+
+
+@pytest.mark.parametrize("case", range(N_BWD_CASES))
+def test_random_backward(fa, case):
+    """dQ, dK, dV of seeded random configurations (head dim 64 or 128, grouped
+    K/V heads, ragged lengths, causal, key padding, Q magnitude) against the
+    oracle's exact gradients, with the backward's bounds."""
+    from tests.test_bwd_gpu import compare_grads, run_bwd
+    rng = np.random.default_rng(777 + 104729 * case)
+    d = int(rng.choice([64, 128]))
+    B = int(rng.integers(1, 3))
+    H_kv = int(rng.integers(1, 4))
+    H = H_kv * int(rng.choice([1, 2, 4]))
+    N = int(rng.integers(1, 600))
+    causal = bool(rng.integers(0, 2))
+    kv_range = (0, N) if rng.random() < 0.4 else None
+    q_mult = float(rng.choice([1.0, 2.0]))
+    import workloads
+    q, k, v, do, kv_len = workloads.make_bwd_inputs(B, H, H_kv, N, d, seed=5000 + case,
+                                                    kv_len_range=kv_range, q_mult=q_mult)
+    what = (f"bwd case {case}: B{B} H{H} H_kv{H_kv} N{N} d{d} causal={causal} "
+            f"kv_len={None if kv_len is None else kv_len.tolist()} q x {q_mult}")
+    got = run_bwd(fa, q, k, v, do, causal, kv_len)
+    ref = oracle.attention_bwd(q, k, v, do, 1.0 / math.sqrt(d), causal=causal, kv_len=kv_len)
+    compare_grads(got, ref, what)
+    print(what + ": ok")
+
+
+N_FP8_CASES = 16
+
+
+@pytest.mark.parametrize("case", range(N_FP8_CASES))
+def test_random_fp8(fa, case):
+    """The e4m3 forward on seeded random configurations (grouped K/V heads,
+    ragged lengths, causal, key padding) against the oracle on the decoded
+    inputs, with the e4m3 bounds."""
+    from tests.test_fp8_gpu import check_fp8
+    rng = np.random.default_rng(31337 + 15485863 * case)
+    B = int(rng.integers(1, 3))
+    H_kv = int(rng.integers(1, 4))
+    H = H_kv * int(rng.choice([1, 2, 4]))
+    N = int(rng.integers(1, 900))
+    causal = bool(rng.integers(0, 2))
+    kv_range = (0, N) if rng.random() < 0.4 else None
+    err = check_fp8(fa, B, H, H_kv, N, causal, seed=7000 + case, kv_len_range=kv_range)
+    print(f"fp8 case {case}: B{B} H{H} H_kv{H_kv} N{N} causal={causal} kv={kv_range}: "
+          f"max|dO|/max|V| {err[0]:.2e}")
