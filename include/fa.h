@@ -134,12 +134,13 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *
 size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits);
 
 /*
- * A num_splits for fa_fwd_splitkv on the current device: the fewest key
- * ranges that give at least 85 % of one wave of work units (one per head group,
- * row block and range) over the SMs, each range at least four 128-key tiles
- * long and at most FA_MAX_SPLITS (every unit pays a fixed cost, so fewer,
- * longer units win once most SMs are busy). Returns 1 for invalid arguments.
- * Reads only device attributes.
+ * A num_splits for fa_fwd_splitkv on the current device: the most key ranges
+ * that keep the work units (one per head group, row block and range) within
+ * one wave over the SMs (units <= SMs), each range at least four 128-key tiles
+ * long and at most FA_MAX_SPLITS; 1 when there are at least as many units as
+ * SMs without splitting (every unit pays a fixed cost, and a second wave leaves
+ * most SMs idle for its last part). Returns 1 for invalid arguments. Reads only
+ * device attributes.
  */
 int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
 
