@@ -293,58 +293,34 @@ __device__ __forceinline__ float row_max(const float (&s)[kTile]) {
 // returns that key's V row to within the output rounding, where O divided by x
 // would carry the dominant probability's rounding (up to 2^-8 of |V|): the
 // reference maximum of a row need not be its true maximum, so its largest
-// probability need not be exactly 1. kPacked = false takes one scalar
-// instruction per score for the scale-subtract and the exact sum instead of
-// one packed (two-lane) instruction per pair: the split-KV form with two
-// accumulators per row, whose packed pairs would spill registers.
-template <int E, bool kPacked = true>
+// probability need not be exactly 1. The scale-subtract and the exact sum
+// take one packed (two-lane fp32) instruction per pair of scores.
+template <int E>
 __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, float mc,
                                            uint32_t tP) {
-    float sum0 = 0.f, sum1 = 0.f;
     if constexpr (E == 2) {
-        if constexpr (kPacked) {
-            float rs0 = 0.f, rs1 = 0.f;
-            float2 sum = make_float2(0.f, 0.f);
-            const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
+        float rs0 = 0.f, rs1 = 0.f;
+        float2 sum = make_float2(0.f, 0.f);
+        const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
 #pragma unroll
-            for (int ch = 0; ch < kTile / 32; ++ch) {
-                uint32_t packed[16];
+        for (int ch = 0; ch < kTile / 32; ++ch) {
+            uint32_t packed[16];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    // The scale-subtract and the exact sum take one packed
-                    // (two-lane fp32) instruction per pair of scores.
-                    const float2 x = __ffma2_rn(
-                        make_float2(s[ch * 32 + 2 * q], s[ch * 32 + 2 * q + 1]), c2, nmc2);
-                    const float p0 = fast_exp2(x.x);
-                    const float p1 = fast_exp2(x.y);
-                    sum = __fadd2_rn(sum, make_float2(p0, p1));
-                    packed[q] = pack_bf16x2(p0, p1);
-                    rs0 = add_bf16_lo(packed[q], rs0);
-                    rs1 = add_bf16_hi(packed[q], rs1);
-                }
-                tmem_st16(tP + (uint32_t)(ch * 16), packed);
+            for (int q = 0; q < 16; ++q) {
+                const float2 x = __ffma2_rn(
+                    make_float2(s[ch * 32 + 2 * q], s[ch * 32 + 2 * q + 1]), c2, nmc2);
+                const float p0 = fast_exp2(x.x);
+                const float p1 = fast_exp2(x.y);
+                sum = __fadd2_rn(sum, make_float2(p0, p1));
+                packed[q] = pack_bf16x2(p0, p1);
+                rs0 = add_bf16_lo(packed[q], rs0);
+                rs1 = add_bf16_hi(packed[q], rs1);
             }
-            return make_float2(sum.x + sum.y, rs0 + rs1);
-        } else {
-            float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < kTile / 32; ++ch) {
-                uint32_t packed[16];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float p0 = fast_exp2(fmaf(s[ch * 32 + 2 * q], c, -mc));
-                    const float p1 = fast_exp2(fmaf(s[ch * 32 + 2 * q + 1], c, -mc));
-                    sum0 += p0;
-                    sum1 += p1;
-                    packed[q] = pack_bf16x2(p0, p1);
-                    rs0 = add_bf16_lo(packed[q], rs0);
-                    rs1 = add_bf16_hi(packed[q], rs1);
-                }
-                tmem_st16(tP + (uint32_t)(ch * 16), packed);
-            }
-            return make_float2(sum0 + sum1, rs0 + rs1);
+            tmem_st16(tP + (uint32_t)(ch * 16), packed);
         }
+        return make_float2(sum.x + sum.y, rs0 + rs1);
     } else {
+        float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
         for (int ch = 0; ch < kTile / 64; ++ch) {
             uint32_t packed[16];
@@ -565,7 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // previous unit's last tiles are consumed, and Q may have to wait.
                 const int early = min(2, 2 * u.n_max);
                 for (int jj = 0; ok && jj < early; ++jj) ok = load_kv(u, jj);
-                for (int t = 0; ok && t < C::kQT; ++t) ok = load_q(t);
+#pragma unroll
+                for (int t = 0; t < C::kQT; ++t) ok = ok && load_q(t);
                 // the rest of K_0, V_0, K_1, V_1, ... of this unit
                 for (int jj = early; ok && jj < 2 * u.n_max; ++jj) ok = load_kv(u, jj);
                 if (!ok) break;
@@ -647,7 +624,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             bool ok = true;
             int L0 = 0;                         // index of this unit's first K/V load
-            uint32_t ph_p[2] = {0u, 0u};        // p_full phases consumed
+            // Per-tile state is indexed by compile-time constants only (the tile
+            // loops are unrolled; one tile keeps bits of one word), so none of
+            // it is placed in local memory.
+            uint32_t ph_p[2] = {0u, 0u};        // p_full phases consumed (two tiles)
+            uint32_t ph_pb = 0u;                // one tile: bit b = parity of p_full[b]'s next phase
             if constexpr (C::kQT == 2) {
             for (int k = 0; ok; ++k) {
                 const int us = k & 1;
@@ -659,13 +640,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const Unit u = decode_unit<C::kQT, kGen>(id, p);
                 // O_t is free once the previous unit's epilogue has read it
                 bool o_ready[2] = {k == 0, k == 0};
-                for (int t = 0; t < 2 && ok; ++t)
-                    ok = mbar_wait(&bars->q_full[t], (uint32_t)(k & 1), wd);
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+                    ok = ok && mbar_wait(&bars->q_full[t], (uint32_t)(k & 1), wd);
                 if (ok && u.n_max > 0) {
                     ok = mbar_wait(&bars->kv_full[L0 % C::kSlots],
                                    (uint32_t)(L0 / C::kSlots) & 1u, wd);
                     if (ok) {
                         tc_fence_after();
+#pragma unroll
                         for (int t = 0; t < 2; ++t) {
                             if (u.n[t] > 0) {
                                 issue_qk(t, t, L0 % C::kSlots);
@@ -682,15 +665,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = mbar_wait(&bars->kv_full[sV], (uint32_t)(LV / C::kSlots) & 1u, wd);
                     if (!ok) break;
                     bool k_ready = false;
-                    for (int t = 0; t < 2 && ok; ++t) {
-                        if (j >= u.n[t]) continue;
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (!ok || j >= u.n[t]) continue;
                         ok = mbar_wait(&bars->p_full[t], ph_p[t] & 1u, wd);
                         ++ph_p[t];
                         if (ok && !o_ready[t]) {
                             ok = mbar_wait(&bars->o_empty[t], (uint32_t)((k - 1) & 1), wd);
                             o_ready[t] = true;
                         }
-                        if (!ok) break;
+                        if (!ok) continue;
                         tc_fence_after();
                         issue_pv(t, t, sV, j > 0);
                         umma_commit(&bars->o_done[t]);
@@ -698,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (!k_ready) {
                                 ok = mbar_wait(&bars->kv_full[sK],
                                                (uint32_t)(LK / C::kSlots) & 1u, wd);
-                                if (!ok) break;
+                                if (!ok) continue;
                                 tc_fence_after();
                                 k_ready = true;
                             }
@@ -712,8 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (k_ready) umma_commit(&bars->kv_empty[sK]);
                 }
                 if (!ok) break;
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (u.n[t] == 0) {                 // idle tile: its once-per-unit hand-offs
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (ok && u.n[t] == 0) {           // idle tile: its once-per-unit hand-offs
                         umma_commit(&bars->q_empty[t]);
                         if (!o_ready[t])
                             ok = mbar_wait(&bars->o_empty[t], (uint32_t)((k - 1) & 1), wd);
@@ -734,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (id < 0) break;
                 const Unit u = decode_unit<C::kQT, kGen>(id, p);
                 const int n = u.n[0];
-                bool o_ready[2] = {k == 0, k == 0};
+                uint32_t o_ready = (k == 0) ? 3u : 0u;   // bit ob: O accumulator ob is free
                 // positions of K_t and V_j in this unit's load order (see the producer)
                 auto posK = [&](int t) { return t < 2 ? t : 2 * t - 1; };
                 auto posV = [&](int j) { return (j <= n - 3) ? 2 + 2 * j : n + j; };
@@ -758,12 +743,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int b = j & 1;
                     ok = wait_load(posV(j));
                     if (!ok) break;
-                    ok = mbar_wait(&bars->p_full[b], ph_p[b] & 1u, wd);
-                    ++ph_p[b];
+                    ok = mbar_wait(&bars->p_full[b], (ph_pb >> b) & 1u, wd);
+                    ph_pb ^= 1u << b;
                     const int ob = kDual ? b : 0;          // O accumulator of this tile
-                    if (ok && !o_ready[ob]) {
+                    if (ok && !((o_ready >> ob) & 1u)) {
                         ok = mbar_wait(&bars->o_empty[ob], (uint32_t)((k - 1) & 1), wd);
-                        o_ready[ob] = true;
+                        o_ready |= 1u << ob;
                     }
                     if (!ok) break;
                     tc_fence_after();
@@ -785,7 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // an O accumulator that took no tile this unit: its once-per-unit hand-offs
                 for (int ob = 0; ok && ob < (kDual ? 2 : 1); ++ob) {
                     if (n > ob) continue;
-                    if (!o_ready[ob])
+                    if (!((o_ready >> ob) & 1u))
                         ok = mbar_wait(&bars->o_empty[ob], (uint32_t)((k - 1) & 1), wd);
                     umma_commit(&bars->o_done[ob]);
                 }
@@ -806,8 +791,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tO = tmem + lane_base + C::col_o(ob);
         const float c = p.scale_log2;
-        uint32_t ph_s[2] = {0u, 0u};   // s_full phases consumed (per S buffer)
-        uint32_t o_base = 0;   // o_done phases of earlier units
+        // Barrier parities, one word: bit b (b = 0, 1) is the parity of s_full[b]'s
+        // next phase, bit 2 that of the o_done phases of earlier units.
+        uint32_t par = 0u;
         bool ok = true;
         for (int k = 0; ok; ++k) {
             const int us = k & 1;
@@ -819,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&bars->unit_empty[us]);
             if (id < 0) break;
             const Unit u = decode_unit<C::kQT, kGen>(id, p);
-            const int n = u.n[t];
+            const int n = t ? u.n[1] : u.n[0];   // a select: an index would put u in local memory
             int row_id;    // (b*H + h)*Nq + i of this thread's row, -1 for a padding row
             int lim_rel;   // visible keys j < lim_rel + kt0*128 (padding rows see none)
             {
@@ -853,7 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto wait_second_last = [&](int j) -> bool {
                 if constexpr (!kDual && C::kQT == 1) {
                     if (j == n - 1 && n >= 2) {
-                        bool w = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(n - 2)) & 1u, wd);
+                        bool w = mbar_wait(&bars->o_done[ob], ((par >> 2) + (uint32_t)(n - 2)) & 1u, wd);
                         return __all_sync(0xffffffffu, w);
                     }
                 }
@@ -864,8 +850,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int jo = kDual ? (j - wg) / 2 : j;       // index among this warpgroup's tiles
                 const int sb = (C::kQT == 2) ? t : (j & 1);   // this tile's S buffer
                 const uint32_t tS = tmem + lane_base + C::col_s(sb);
-                ok = mbar_wait(&bars->s_full[sb], ph_s[sb] & 1u, wd);
-                ++ph_s[sb];
+                ok = mbar_wait(&bars->s_full[sb], (par >> sb) & 1u, wd);
+                par ^= 1u << sb;
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 if (idle_warp) {
@@ -918,14 +904,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // them (P of this tile is not handed over yet, so o_done is
                         // exactly at that phase or one short), then rescale it, 16
                         // columns at a time while the tile's scores are live.
-                        ok = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(jo - 1)) & 1u, wd);
+                        ok = mbar_wait(&bars->o_done[ob], ((par >> 2) + (uint32_t)(jo - 1)) & 1u, wd);
                         ok = __all_sync(0xffffffffu, ok);
                         if (!ok) break;
                         tc_fence_after();
                         rescale_o<D, 16>(tO, alpha);
                     }
                     const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-                    l_tile = exp_tile<E, !kDual>(s, c, mc, tS);
+                    l_tile = exp_tile<E>(s, c, mc, tS);
                     l += l_tile.x;
                     lr += l_tile.y;
                 } else {
@@ -938,7 +924,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // fp32 and bf16 range, and O / l is exact whatever m_ref is.
                     if (m_ref == -INFINITY) m_ref = row_max(s);
                     float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-                    l_tile = exp_tile<E, !kDual>(s, c, mc, tS);
+                    l_tile = exp_tile<E>(s, c, mc, tS);
                     const bool stale = !(l_tile.x <= redo_tile_sum<E>());
                     if (__any_sync(0xffffffffu, stale)) {
                         if (stale) {
@@ -950,14 +936,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             rescale = true;
                         }
                         mc = m_ref * c;
-                        l_tile = exp_tile<E, !kDual>(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
+                        l_tile = exp_tile<E>(s, c, mc, tS);   // tcgen05.st is warp-wide: redo all rows
                     }
                     l += l_tile.x;
                     lr += l_tile.y;
                     if (__any_sync(0xffffffffu, rescale)) {
                         // O holds the P.V sums of tiles < j: wait for the last of
                         // them, then bring it to the new reference maximum.
-                        ok = mbar_wait(&bars->o_done[ob], (o_base + (uint32_t)(jo - 1)) & 1u, wd);
+                        ok = mbar_wait(&bars->o_done[ob], ((par >> 2) + (uint32_t)(jo - 1)) & 1u, wd);
                         ok = __all_sync(0xffffffffu, ok);
                         if (!ok) break;
                         tc_fence_after();
@@ -974,8 +960,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // ------------------------------------------------ epilogue
             // the unit's last o_done phase for this accumulator (its idle phase if none)
-            const uint32_t last = o_base + (uint32_t)(n_own > 0 ? n_own - 1 : 0);
-            o_base += (uint32_t)(n_own > 0 ? n_own : 1);
+            const uint32_t last = (par >> 2) + (uint32_t)(n_own > 0 ? n_own - 1 : 0);
+            par ^= (uint32_t)((n_own > 0 ? n_own : 1) & 1) << 2;
             ok = mbar_wait(&bars->o_done[ob], last & 1u, wd);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
