@@ -156,12 +156,26 @@ int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
  * e4m3 with fp32 accumulation, and the probabilities P are rounded to e4m3
  * (relative error up to 2^-4) before the P.V product, so O carries that
  * error; lse does not (scores are exact products of e4m3 values). d must be
- * 128 (else FA_ERR_UNSUPPORTED); causal, kv_len, H_kv, errors as in
+ * 128 or 256 (d = 64: FA_ERR_UNSUPPORTED); causal, kv_len, H_kv, errors as in
  * fa_fwd_gqa.
  */
 int fa_fwd_fp8(const void *q, const void *k, const void *v, float q_descale, float k_descale,
                float v_descale, void *o, float *lse, int B, int H, int H_kv, int N, int d,
                float scale, int causal, const int32_t *kv_len, void *stream);
+
+/*
+ * FP8 split-KV forward: fa_fwd_splitkv with e4m3 q [B, H, Nq, d] and k, v
+ * [B, H_kv, Nk, d] and their descales as in fa_fwd_fp8 (same precision
+ * statement). O bf16 [B, H, Nq, d], lse fp32 [B, H, Nq]; the partials in
+ * `workspace` are fp32, sized by fa_splitkv_workspace_bytes as for bf16
+ * inputs. d must be 128 or 256 (d = 64: FA_ERR_UNSUPPORTED); every other
+ * argument and error as in fa_fwd_splitkv.
+ */
+int fa_fwd_splitkv_fp8(const void *q, const void *k, const void *v, float q_descale,
+                       float k_descale, float v_descale, void *o, float *lse, int B, int H,
+                       int H_kv, int Nq, int Nk, int d, float scale, int causal,
+                       const int32_t *kv_len, int num_splits, void *workspace,
+                       size_t workspace_bytes, void *stream);
 
 /*
  * Backward pass: gradients of the attention of fa_fwd / fa_fwd_gqa for a

@@ -66,6 +66,9 @@ def load_library(path: str = LIB_PATH):
     lib.fa_fwd_splitkv_static.restype = i
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, i, vp, vp]
     lib.fa_fwd_fp8.restype = i
+    lib.fa_fwd_splitkv_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, i, f, i, vp,
+                                       i, vp, sz, vp]
+    lib.fa_fwd_splitkv_fp8.restype = i
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp,
                            sz, vp]
     lib.fa_bwd.restype = i
@@ -145,6 +148,16 @@ def fa_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, B, H, H_kv, N, 
     """C ABI fa_fwd_fp8: e4m3 q, k, v with per-tensor descales; bf16 O, fp32 lse."""
     return load_library().fa_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, B, H,
                                      H_kv, N, d, scale, causal, kv_len, stream)
+
+
+def fa_fwd_splitkv_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, B, H, H_kv, Nq, Nk,
+                       d, scale, causal, kv_len, num_splits, workspace, workspace_bytes,
+                       stream) -> int:
+    """C ABI fa_fwd_splitkv_fp8: the split-KV forward on e4m3 q, k, v with
+    per-tensor descales; bf16 O, fp32 lse."""
+    return load_library().fa_fwd_splitkv_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse,
+                                             B, H, H_kv, Nq, Nk, d, scale, causal, kv_len,
+                                             num_splits, workspace, workspace_bytes, stream)
 
 
 def fa_bwd(q, k, v, o, lse, d_o, dq, dk, dv, B, H, H_kv, N, d, scale, causal, kv_len,
@@ -330,4 +343,45 @@ def attention_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causa
                     int(bool(causal)), _ptr(kv_len), s)
     if check and st != FA_OK:
         raise FAError(st, "fa_fwd_fp8")
+    return out, lse
+
+
+def decode_attention_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None,
+                         causal=False, kv_len=None, num_splits=None, out=None, lse=None,
+                         workspace=None, stream=None, check=True):
+    """O (bf16), lse for e4m3 CUDA tensors q8 [B, H, Nq, d] and k8, v8
+    [B, H_kv, Nk, d] (Nq <= Nk) with per-tensor descales, through
+    fa_fwd_splitkv_fp8 (key ranges merged by their log-sum-exp)."""
+    import torch
+    for t in (q8, k8, v8):
+        if t.element_size() != 1 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q8, k8, v8 must be contiguous one-byte CUDA tensors")
+    if q8.dim() != 4 or k8.dim() != 4 or k8.shape != v8.shape or \
+            (q8.shape[0], q8.shape[3]) != (k8.shape[0], k8.shape[3]):
+        raise ValueError(f"q [B,H,Nq,d] and k, v [B,H_kv,Nk,d] expected, got "
+                         f"{q8.shape} {k8.shape} {v8.shape}")
+    B, H, Nq, d = q8.shape
+    H_kv, Nk = k8.shape[1], k8.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if num_splits is None:
+        num_splits = fa_splitkv_default_splits(B, H, H_kv, Nq, Nk, d)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
+    if kv_len is not None and (kv_len.dtype != torch.int32 or not kv_len.is_cuda
+                               or kv_len.shape != (B,)):
+        raise ValueError("kv_len must be a CUDA int32 tensor of shape [B]")
+    need = fa_splitkv_workspace_bytes(B, H, Nq, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q8.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    s = stream if stream is not None else torch.cuda.current_stream(q8.device).cuda_stream
+    st = fa_fwd_splitkv_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_descale), float(k_descale),
+                            float(v_descale), _ptr(out), _ptr(lse), B, H, H_kv, Nq, Nk, d,
+                            float(scale), int(bool(causal)), _ptr(kv_len), int(num_splits),
+                            _ptr(workspace), ws_bytes, s)
+    if check and st != FA_OK:
+        raise FAError(st, "fa_fwd_splitkv_fp8")
     return out, lse

@@ -108,7 +108,9 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
             const bool ok = set_smem<64, 2, false>() && set_smem<128, 2, false>() &&
                             set_smem<256, 1, false>() && set_smem<64, 1, true>() &&
                             set_smem<128, 1, true>() && set_smem<256, 1, true>() &&
-                            set_smem<128, 2, false, 1>() && set_bwd_smem<64>() &&
+                            set_smem<128, 2, false, 1>() && set_smem<256, 1, false, 1>() &&
+                            set_smem<128, 1, true, 1>() && set_smem<256, 1, true, 1>() &&
+                            set_bwd_smem<64>() &&
                             set_bwd_smem<128>();
             if (!ok) return FA_ERR_LAUNCH;
         }
@@ -254,7 +256,7 @@ int fwd_check(const FwdCall& a, FwdPlan* pl) {
     if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     const int E = a.elem;
     if (E == 1) {
-        if (d != 128) return FA_ERR_UNSUPPORTED;
+        if (d == 64) return FA_ERR_UNSUPPORTED;   // e4m3: d = 128 or 256
         for (float x : {a.q_descale, a.k_descale, a.v_descale})
             if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
     }
@@ -278,7 +280,6 @@ int fwd_check(const FwdCall& a, FwdPlan* pl) {
     // Square attention (one key range, no packing, Nq == Nk) runs the
     // specialised kernels; everything else the general one-query-tile kernel.
     pl->general = a.splits > 1 || pl->G > 1 || Nq != Nk;
-    if (E == 1 && pl->general) return FA_ERR_UNSUPPORTED;   // e4m3: square attention only
     pl->qt = (pl->general || d == 256) ? 1 : 2;              // query tiles per unit
     const int64_t n_rb = ((int64_t)Nq + pl->nq_blk - 1) / pl->nq_blk;
     pl->n_units = (n_rb + pl->qt - 1) / pl->qt * a.splits;    // <= 2^31 * 128
@@ -369,7 +370,14 @@ int fwd_impl(const FwdCall& a, void* stream) {
     const dim3 grid((unsigned)(BHB * n_units)), block(kThreads);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (E == 1) {
-        fa_fwd_sm100<128, 2, false, 1><<<grid, block, Cfg<128, 2, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        if (pl.general && d == 256)
+            fa_fwd_sm100<256, 1, true, 1><<<grid, block, Cfg<256, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else if (pl.general)
+            fa_fwd_sm100<128, 1, true, 1><<<grid, block, Cfg<128, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else if (d == 256)
+            fa_fwd_sm100<256, 1, false, 1><<<grid, block, Cfg<256, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else
+            fa_fwd_sm100<128, 2, false, 1><<<grid, block, Cfg<128, 2, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
     } else if (pl.general) {
         if (d == 256)
             fa_fwd_sm100<256, 1, true><<<grid, block, Cfg<256, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
@@ -632,6 +640,23 @@ FA_EXPORT int fa_fwd_fp8(const void* q, const void* k, const void* v, float q_de
                          int H_kv, int N, int d, float scale, int causal,
                          const int32_t* kv_len, void* stream) {
     fa::FwdCall a = fa::square_call(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, kv_len);
+    a.elem = 1;
+    a.q_descale = q_descale;
+    a.k_descale = k_descale;
+    a.v_descale = v_descale;
+    return fa::fwd_impl(a, stream);
+}
+
+FA_EXPORT int fa_fwd_splitkv_fp8(const void* q, const void* k, const void* v, float q_descale,
+                                 float k_descale, float v_descale, void* o, float* lse, int B,
+                                 int H, int H_kv, int Nq, int Nk, int d, float scale, int causal,
+                                 const int32_t* kv_len, int num_splits, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    fa::FwdCall a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.H = H; a.H_kv = H_kv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+    a.scale = scale; a.causal = causal; a.kv_len = kv_len;
+    a.splits = num_splits; a.pack = true; a.ws = workspace; a.ws_bytes = workspace_bytes;
     a.elem = 1;
     a.q_descale = q_descale;
     a.k_descale = k_descale;

@@ -107,19 +107,20 @@ constexpr float kLn2 = 0.69314718055994530942f;
 // current ones. d = 256 needs it (O alone takes 256 TMEM columns); the
 // split-KV kernel uses it at every d, since a short query block gives the
 // second tile of a pair nothing to do.
-// E is the element size of Q, K and V: 2 (bf16) or 1 (e4m3, d = 128 only).
+// E is the element size of Q, K and V: 2 (bf16) or 1 (e4m3, d = 128 or 256:
+// a 64-byte row at d = 64 would need another swizzle layout).
 template <int D, int QT, int E = 2>
 struct Cfg {
     static_assert(D == 64 || D == 128 || D == 256, "head dim 64, 128 or 256");
     static_assert(QT == 1 || (QT == 2 && D <= 128), "two query tiles need d <= 128");
-    static_assert(E == 2 || (E == 1 && D == 128), "e4m3 inputs need d = 128");
+    static_assert(E == 2 || (E == 1 && D >= 128), "e4m3 inputs need d = 128 or 256");
     static constexpr int kQT = QT;                        // query tiles per unit
     static constexpr int kBlocks = D * E / 128;           // 128-byte column blocks per row
     static constexpr int kBlockElems = 128 / E;           // columns of one block
     static constexpr int kBlockBytes = kTile * 128;       // 16 KB
     static constexpr int kTileBytes = kTile * D * E;      // one Q/K/V tile
     static constexpr int kSlots =                         // K/V ring depth
-        (E == 1) ? 8 : (D == 256) ? 2 : (D == 128) ? (QT == 2 ? 4 : 5) : 8;
+        (D * E == 256) ? (QT == 2 ? 4 : 5) : (D * E == 512) ? 2 : 8;
     static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 4096 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
@@ -320,39 +321,43 @@ __device__ __forceinline__ float2 exp_tile(const float (&s)[kTile], float c, flo
         }
         return make_float2(sum.x + sum.y, rs0 + rs1);
     } else {
-        float sum0 = 0.f, sum1 = 0.f;
+        float2 sum = make_float2(0.f, 0.f);
+        const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
 #pragma unroll
         for (int ch = 0; ch < kTile / 64; ++ch) {
             uint32_t packed[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-                float pq[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pq[e] = fast_exp2(fmaf(s[ch * 64 + 4 * q + e], c, -mc));
-                sum0 += pq[0] + pq[2];
-                sum1 += pq[1] + pq[3];
-                packed[q] = pack_e4m3x4(pq[0], pq[1], pq[2], pq[3]);
+                const float* sq = &s[ch * 64 + 4 * q];
+                const float2 x0 = __ffma2_rn(make_float2(sq[0], sq[1]), c2, nmc2);
+                const float2 x1 = __ffma2_rn(make_float2(sq[2], sq[3]), c2, nmc2);
+                const float p0 = fast_exp2(x0.x), p1 = fast_exp2(x0.y);
+                const float p2 = fast_exp2(x1.x), p3 = fast_exp2(x1.y);
+                sum = __fadd2_rn(sum, __fadd2_rn(make_float2(p0, p1), make_float2(p2, p3)));
+                packed[q] = pack_e4m3x4(p0, p1, p2, p3);
             }
             tmem_st16(tP + (uint32_t)(ch * 16), packed);
         }
-        return make_float2(sum0 + sum1, sum0 + sum1);
+        return make_float2(sum.x + sum.y, sum.x + sum.y);
     }
 }
 
-// Two query tiles: a row's reference maximum is raised only when a tile's
-// maximum exceeds it by more than this (log2 units), so every probability is
-// at most 2^64 for bf16 P, or 2^8 for e4m3 P, whose largest finite value is 448.
+// Max-first rule (two query tiles, and e4m3 at any tile count): a row's
+// reference maximum is raised only when a tile's maximum exceeds it by more
+// than this (log2 units), so every probability is at most 2^64 for bf16 P, or
+// 2^8 for e4m3 P, whose largest finite value is 448.
 template <int E>
 __device__ __forceinline__ constexpr float rescale_log2() {
     return E == 2 ? 64.0f : 8.0f;
 }
 
-// One query tile: the largest row sum of a tile's probabilities, computed
-// against the reference, before the row takes its true maximum and the tile is
-// redone (2^64 for bf16 P).
+// Exponentiate-first rule (one bf16 query tile): the largest row sum of a
+// tile's probabilities, computed against the reference, before the row takes
+// its true maximum and the tile is redone (2^64).
 template <int E>
 __device__ __forceinline__ constexpr float redo_tile_sum() {
-    return E == 2 ? 18446744073709551616.0f : 256.0f;
+    static_assert(E == 2, "e4m3 takes the max-first rule");
+    return 18446744073709551616.0f;
 }
 
 // O (d columns of this thread's TMEM lane) *= alpha, kCols columns at a time.
@@ -401,9 +406,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kConsumers = 1 + kSoftmaxWarps;   // MMA thread + one lane per softmax warp
     // Reference-maximum rule (see the softmax loop): fixed before the
     // exponentials with two query tiles, where it measured faster; exponentiate
-    // first and redo the rare overshooting tile with one (S double-buffered, the
-    // row maximum pass would sit on the critical path).
-    constexpr bool kMaxFirst = QT == 2;
+    // first and redo the rare overshooting tile with one bf16 tile (S
+    // double-buffered, the row maximum pass would sit on the critical path).
+    // e4m3 P allows an overshoot of 2^8 only, so a redo would not be rare: e4m3
+    // takes the max-first rule at every tile count.
+    constexpr bool kMaxFirst = QT == 2 || E == 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -601,8 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             };
             // O of tile t (+)= P in S buffer sb . V tile in `slot`. At d = 256 each
-            // K-step is issued as two N = 128 MMAs, one per half of V's column
-            // blocks (the same instruction shape as d = 128).
+            // K-step is issued as two N = 128 MMAs, one per half of V's columns
+            // (the same instruction shape as d = 128): two 128-byte column
+            // blocks of bf16, one of e4m3.
             auto issue_pv = [&](int t, int sb, int slot, bool accumulate) {
                 const uint64_t b = dv0 + (uint64_t)slot * kTileStep;
                 const uint32_t tP = tmem + C::col_s(sb);
@@ -611,14 +619,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int h = 0; h < kPvHalves; ++h) {
                         const uint64_t bk = b + (uint64_t)((kk * kStepRows * 128 +
-                                                            h * (kPvN / 64) * C::kBlockBytes) >> 4);
+                                                            h * (kPvN * E / 128) * C::kBlockBytes) >> 4);
                         if constexpr (E == 2)
                             umma_ts(tmem + C::col_o(t) + (uint32_t)(h * kPvN),
                                     tP + (uint32_t)(kk * 8), bk, idesc_pv,
                                     (accumulate || kk > 0) ? 1u : 0u);
                         else
-                            umma_ts_f8(tmem + C::col_o(t), tP + (uint32_t)(kk * 8),
-                                       bk, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                            umma_ts_f8(tmem + C::col_o(t) + (uint32_t)(h * kPvN),
+                                       tP + (uint32_t)(kk * 8), bk, idesc_pv,
+                                       (accumulate || kk > 0) ? 1u : 0u);
                     }
                 }
             };

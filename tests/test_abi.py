@@ -19,7 +19,8 @@ def lib():
 def test_header_declares_the_boundary():
     assert fa.declared_symbols() == ["fa_bwd", "fa_bwd_workspace_bytes",
                                      "fa_fwd", "fa_fwd_fp8", "fa_fwd_gqa", "fa_fwd_kvlen",
-                                     "fa_fwd_splitkv", "fa_fwd_splitkv_static",
+                                     "fa_fwd_splitkv", "fa_fwd_splitkv_fp8",
+                                     "fa_fwd_splitkv_static",
                                      "fa_last_device_error",
                                      "fa_splitkv_default_splits",
                                      "fa_splitkv_workspace_bytes", "fa_status_string",
@@ -221,7 +222,7 @@ def test_bwd_workspace_bytes(lib):
 # ---------------------------------------------------------------- e4m3 forward
 @pytest.mark.parametrize("over,status", [
     (dict(d=64), fa.FA_ERR_UNSUPPORTED),
-    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=32), fa.FA_ERR_UNSUPPORTED),
     (dict(qs=0.0), fa.FA_ERR_INVALID_ARG),
     (dict(ks=-1.0), fa.FA_ERR_INVALID_ARG),
     (dict(vs=float("inf")), fa.FA_ERR_INVALID_ARG),
@@ -239,3 +240,31 @@ def test_fp8_argument_errors_are_synchronous(lib, over, status):
                         a["B"], a["H"], a["H_kv"], a["N"], a["d"], a["scale"], a["causal"],
                         None, None)
     assert st == status
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(d=64), fa.FA_ERR_UNSUPPORTED),
+    (dict(qs=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(vs=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(Nq=513), fa.FA_ERR_INVALID_ARG),            # more queries than keys
+    (dict(splits=0), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=129), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=None), fa.FA_ERR_INVALID_ARG),           # splits > 1 needs a workspace
+    (dict(ws_bytes=16), fa.FA_ERR_INVALID_ARG),       # too small
+    (dict(ws=P + (5 << 30) + 8), fa.FA_ERR_INVALID_ARG),   # misaligned
+    (dict(ws=P), fa.FA_ERR_INVALID_ARG),              # overlaps q
+    (dict(B=0), fa.FA_OK),
+])
+def test_fp8_splitkv_argument_errors_are_synchronous(lib, over, status):
+    """The e4m3 split-KV entry checks its arguments like fa_fwd_splitkv and
+    fa_fwd_fp8, before any CUDA call."""
+    a = dict(q=P, k=P + (1 << 30), v=P + (2 << 30), o=P + (3 << 30), lse=P + (4 << 30),
+             ws=P + (5 << 30), ws_bytes=1 << 29, qs=0.01, ks=0.01, vs=0.01, B=2, H=8, H_kv=2,
+             Nq=4, Nk=512, d=128, scale=0.088, causal=1, splits=3)
+    a.update(over)
+    st = lib.fa_fwd_splitkv_fp8(a["q"], a["k"], a["v"], a["qs"], a["ks"], a["vs"], a["o"],
+                                a["lse"], a["B"], a["H"], a["H_kv"], a["Nq"], a["Nk"], a["d"],
+                                a["scale"], a["causal"], None, a["splits"], a["ws"],
+                                a["ws_bytes"], None)
+    assert st == status
+

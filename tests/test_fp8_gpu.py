@@ -1,5 +1,6 @@
-"""GPU parity of the e4m3 forward (fa_fwd_fp8) against the fp64 oracle on the
-dequantized inputs (oracle.fp8.attention_fp8).
+"""GPU parity of the e4m3 forward (fa_fwd_fp8 at d = 128 and 256, and the
+split-KV form fa_fwd_splitkv_fp8) against the fp64 oracle on the dequantized
+inputs (oracle.fp8.attention_fp8).
 
 Tolerance, derived from the arithmetic: scores are exact (products of e4m3
 values are exact in fp32; accumulation is fp32), so lse keeps the bf16 path's
@@ -32,14 +33,20 @@ def fa():
     return fa
 
 
-def run_fp8(fa, q8, k8, v8, sc, causal, kv_len=None):
+def run_fp8(fa, q8, k8, v8, sc, causal, kv_len=None, cache=False, splits=None):
+    """One e4m3 launch: square (fa_fwd_fp8) or, with cache=True, through the
+    split-KV entry (Nq <= Nk, query heads of a K/V group packed)."""
     dev = torch.device("cuda:0")
     qd, kd, vd = (x.to(dev) for x in (q8, k8, v8))
     kvd = None if kv_len is None else kv_len.to(dev)
     B, H, N, d = q8.shape
     out = torch.full((B, H, N, d), float("nan"), dtype=torch.bfloat16, device=dev)
     lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
-    fa.attention_fp8(qd, kd, vd, *sc, causal=causal, kv_len=kvd, out=out, lse=lse)
+    if cache:
+        fa.decode_attention_fp8(qd, kd, vd, *sc, causal=causal, kv_len=kvd,
+                                num_splits=splits, out=out, lse=lse)
+    else:
+        fa.attention_fp8(qd, kd, vd, *sc, causal=causal, kv_len=kvd, out=out, lse=lse)
     st = fa.fa_last_device_error(torch.cuda.current_stream().cuda_stream)
     assert st == fa.FA_OK, fa.fa_status_string(st)
     return out.double().cpu().numpy(), lse.double().cpu().numpy()
@@ -61,13 +68,20 @@ def compare_fp8(o, lse, o_ref, lse_ref, vmax, what, rows=None):
     return float(err.max() / vmax), float(err.mean() / vmax)
 
 
-def check_fp8(fa, B, H, H_kv, N, causal, seed, kv_len_range=None, rows=None):
-    q8, k8, v8, sc, kvl = workloads.make_fp8_inputs(B, H, H_kv, N, 128, seed, kv_len_range)
-    o, lse = run_fp8(fa, q8, k8, v8, sc, causal, kvl)
-    o_ref, lse_ref = ofp8.attention_fp8(q8, k8, v8, *sc, 1.0 / math.sqrt(128), causal=causal,
+def check_fp8(fa, B, H, H_kv, N, causal, seed, kv_len_range=None, rows=None, d=128,
+              Nk=None, splits=None):
+    """Parity of one e4m3 configuration. Nk given: the split-KV entry with N
+    query rows against Nk keys (splits key ranges, None for the library's
+    choice); else the square entry."""
+    cache = Nk is not None
+    q8, k8, v8, sc, kvl = workloads.make_fp8_inputs(B, H, H_kv, N, d, seed, kv_len_range,
+                                                    Nk=Nk)
+    o, lse = run_fp8(fa, q8, k8, v8, sc, causal, kvl, cache=cache, splits=splits)
+    o_ref, lse_ref = ofp8.attention_fp8(q8, k8, v8, *sc, 1.0 / math.sqrt(d), causal=causal,
                                         kv_len=kvl, rows=rows)
     vmax = float(np.abs(ofp8.decode_e4m3(v8.view(torch.uint8).numpy())).max() * sc[2])
-    return compare_fp8(o, lse, o_ref, lse_ref, vmax, f"B{B} H{H}/{H_kv} N{N} c{causal}", rows)
+    what = f"B{B} H{H}/{H_kv} N{N} Nk{Nk} d{d} c{causal} splits={splits}"
+    return compare_fp8(o, lse, o_ref, lse_ref, vmax, what, rows)
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -94,3 +108,42 @@ def test_fp8_is_deterministic(fa):
     a = run_fp8(fa, q8, k8, v8, sc, True)
     b = run_fp8(fa, q8, k8, v8, sc, True)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 129, 300, 1024])
+def test_fp8_head_dim_256(fa, N, causal):
+    """d = 256: one query tile per unit, two 128-byte column blocks per row."""
+    check_fp8(fa, 2, 2, 2, N, causal, seed=6400 + N + causal, d=256)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_head_dim_256_grouped_heads_and_padding(fa, causal):
+    check_fp8(fa, 2, 4, 2, 600, causal, seed=6500 + causal, kv_len_range=(0, 600), d=256)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("Nq,Nk,H,H_kv,splits,causal", [
+    (1, 4096, 8, 2, None, False),       # one-token decoding, the library's key ranges
+    (1, 1000, 4, 4, 3, True),           # ragged key count, three ranges
+    (16, 777, 8, 1, 2, True),           # multi-query: 8 heads packed, 16 rows each
+    (200, 200, 4, 2, 1, True),          # Nq == Nk through the general kernel
+    (130, 2048, 2, 1, 5, False),        # two row blocks per head pair
+])
+def test_fp8_splitkv(fa, d, Nq, Nk, H, H_kv, splits, causal):
+    """The e4m3 split-KV entry: Nq <= Nk with the causal offset Nk - Nq,
+    grouped heads packed into one tile, key ranges merged by their lse."""
+    check_fp8(fa, 2, H, H_kv, Nq, causal, seed=6600 + Nq + d, d=d, Nk=Nk, splits=splits)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_fp8_splitkv_key_padding(fa, d):
+    """kv_len per batch (0 included: empty rows give lse = -inf and O = 0)."""
+    q8, k8, v8, sc, _ = workloads.make_fp8_inputs(3, 4, 2, 5, d, 6700 + d, Nk=900)
+    kvl = torch.tensor([0, 1, 637], dtype=torch.int32)
+    o, lse = run_fp8(fa, q8, k8, v8, sc, False, kvl, cache=True, splits=4)
+    o_ref, lse_ref = ofp8.attention_fp8(q8, k8, v8, *sc, 1.0 / math.sqrt(d), kv_len=kvl)
+    vmax = float(np.abs(ofp8.decode_e4m3(v8.view(torch.uint8).numpy())).max() * sc[2])
+    compare_fp8(o, lse, o_ref, lse_ref, vmax, f"kv_len padding d{d}")
+    assert np.all(o[0] == 0.0) and np.all(np.isneginf(lse[0]))
+

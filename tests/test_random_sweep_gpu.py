@@ -133,3 +133,33 @@ def test_random_fp8(fa, case):
     err = check_fp8(fa, B, H, H_kv, N, causal, seed=7000 + case, kv_len_range=kv_range)
     print(f"fp8 case {case}: B{B} H{H} H_kv{H_kv} N{N} causal={causal} kv={kv_range}: "
           f"max|dO|/max|V| {err[0]:.2e}")
+
+
+N_FP8_MORE = 16
+
+
+@pytest.mark.parametrize("case", range(N_FP8_MORE))
+def test_random_fp8_d256_and_cache(fa, case):
+    """The e4m3 forward at d = 256 (square) and through the split-KV entry at
+    d = 128 and 256 (fewer query rows than keys, packed heads, key ranges) on
+    seeded random configurations, with the e4m3 bounds."""
+    from tests.test_fp8_gpu import check_fp8
+    rng = np.random.default_rng(4242 + 7919 * case)
+    B = int(rng.integers(1, 3))
+    H_kv = int(rng.integers(1, 3))
+    H = H_kv * int(rng.choice([1, 2, 4, 8]))
+    causal = bool(rng.integers(0, 2))
+    if case % 2 == 0:
+        d, N = 256, int(rng.integers(1, 700))
+        Nk, splits = None, None
+    else:
+        d = int(rng.choice([128, 256]))
+        Nk = int(rng.integers(1, 1500))
+        N = int(rng.integers(1, min(Nk, 200) + 1))
+        splits = [None, 1, 2, 5][int(rng.integers(0, 4))]
+    kv_hi = N if Nk is None else Nk
+    kv_range = (0, kv_hi) if rng.random() < 0.4 else None
+    err = check_fp8(fa, B, H, H_kv, N, causal, seed=7100 + case, kv_len_range=kv_range, d=d,
+                    Nk=Nk, splits=splits)
+    print(f"fp8 case {case}: B{B} H{H} H_kv{H_kv} N{N} Nk{Nk} d{d} causal={causal} "
+          f"splits={splits} kv={kv_range}: max|dO|/max|V| {err[0]:.2e}")

@@ -209,15 +209,17 @@ def make_bwd_inputs(B, H, H_kv, N, d, seed, kv_len_range=None, q_mult=1.0):
     return q, k, v, do, kv_len
 
 
-def make_fp8_inputs(B, H, H_kv, N, d, seed, kv_len_range=None):
+def make_fp8_inputs(B, H, H_kv, N, d, seed, kv_len_range=None, Nk=None):
     """e4m3 inputs: the same draws as make_inputs (Q, then K, then V, N(0,1)
     fp32), each divided by its descale amax / 448 and rounded to e4m3 by
     torch's float8_e4m3fn conversion (round to nearest even, no saturation
-    needed). Returns (q8, k8, v8, (q_descale, k_descale, v_descale), kv_len)."""
+    needed). q has N rows, k and v Nk (default N) keys. Returns (q8, k8, v8,
+    (q_descale, k_descale, v_descale), kv_len)."""
+    Nk = N if Nk is None else Nk
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     xs = [torch.randn(shape, generator=g, dtype=torch.float32)
-          for shape in ((B, H, N, d), (B, H_kv, N, d), (B, H_kv, N, d))]
+          for shape in ((B, H, N, d), (B, H_kv, Nk, d), (B, H_kv, Nk, d))]
     kv_len = None
     if kv_len_range is not None:
         lo, hi = kv_len_range
