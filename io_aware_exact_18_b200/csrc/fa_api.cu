@@ -13,6 +13,7 @@
 #include "fa.h"
 #include "fa_bwd_kernel.cuh"
 #include "fa_combine_kernel.cuh"
+#include "fa_decode_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
@@ -71,6 +72,12 @@ bool set_smem() {
                                 Cfg<D, QT, E>::kSmemBytes) == cudaSuccess;
 }
 
+template <int D>
+bool set_decode_smem() {
+    return cudaFuncSetAttribute(fa_decode_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                DecCfg<D>::kSmemBytes) == cudaSuccess;
+}
+
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
@@ -110,6 +117,7 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
                             set_smem<128, 1, true>() && set_smem<256, 1, true>() &&
                             set_smem<128, 2, false, 1>() && set_smem<256, 1, false, 1>() &&
                             set_smem<128, 1, true, 1>() && set_smem<256, 1, true, 1>() &&
+                            set_decode_smem<128>() &&
                             set_bwd_smem<64>() &&
                             set_bwd_smem<128>();
             if (!ok) return FA_ERR_LAUNCH;
@@ -369,7 +377,14 @@ int fwd_impl(const FwdCall& a, void* stream) {
 
     const dim3 grid((unsigned)(BHB * n_units)), block(kThreads);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (E == 1) {
+    // Decoding shapes (bf16, d = 128, a K/V group's query heads times the query
+    // rows within kDecLive columns: one row block per group) take the
+    // transposed tile; the unit grid is the same (head group, range) set.
+    const bool dec = E == 2 && d == 128 && pl.general && Nq == nq_blk &&
+                     (int64_t)G * Nq <= kDecLive && G == H / H_kv;
+    if (dec) {
+        fa_decode_sm100<128><<<grid, dim3(kDecThreads), DecCfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
+    } else if (E == 1) {
         if (pl.general && d == 256)
             fa_fwd_sm100<256, 1, true, 1><<<grid, block, Cfg<256, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
         else if (pl.general)
