@@ -136,11 +136,12 @@ size_t fa_splitkv_workspace_bytes(int B, int H, int Nq, int d, int num_splits);
 /*
  * A num_splits for fa_fwd_splitkv on the current device: the most key ranges
  * that keep the work units (one per head group, row block and range) within
- * one wave over the SMs (units <= SMs), each range at least four 128-key tiles
- * long and at most FA_MAX_SPLITS; 1 when there are at least as many units as
- * SMs without splitting (every unit pays a fixed cost, and a second wave leaves
- * most SMs idle for its last part). Returns 1 for invalid arguments. Reads only
- * device attributes.
+ * one wave, units <= the device's SM count, or <= 128 for the decoding tile
+ * (bf16, d = 128, at most 8 query heads x rows per K/V head), which measured
+ * fastest there; each range at least four 128-key tiles long and at most
+ * FA_MAX_SPLITS; 1 when there are at least that many units without splitting
+ * (every unit pays a fixed cost, and a second wave leaves most SMs idle for its
+ * last part). Returns 1 for invalid arguments. Reads only device attributes.
  */
 int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
 

@@ -125,6 +125,10 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
         st.probed = true;
     }
     if (!st.supported) return FA_ERR_UNSUPPORTED;
+    // Launch failures are read back through cudaGetLastError: clear an error
+    // an earlier, unrelated runtime call may have left there (a sticky error
+    // stays and fails the launch anyway).
+    (void)cudaGetLastError();
     *dev_out = dev;
     *err_out = st.err_ptr;
     return FA_OK;
@@ -410,19 +414,35 @@ int fwd_impl(const FwdCall& a, void* stream) {
     }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
     if (a.splits > 1) {
-        const dim3 cgrid((unsigned)((rows + kCombineWarps - 1) / kCombineWarps));
-        const dim3 cblock(32 * kCombineWarps);
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)((rows + kCombineWarps - 1) / kCombineWarps));
+        cfg.blockDim = dim3(32 * kCombineWarps);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        // After the decoding kernel (not persistent; each CTA signals once it
+        // has started) the merge is a programmatic dependent: its launch
+        // overlaps the decoding grid's tail and it waits for that grid's
+        // completion before reading the partials.
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = dec ? 1 : 0;
         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
+        cudaError_t e;
         if (d == 256)
-            fa_splitkv_combine<256><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits,
-                                                              err);
+            e = cudaLaunchKernelEx(&cfg, fa_splitkv_combine<256>, (const float*)o_part,
+                                   (const float*)lse_part, o, a.lse, (int64_t)rows, a.splits,
+                                   (const uint32_t*)err);
         else if (d == 128)
-            fa_splitkv_combine<128><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits,
-                                                              err);
+            e = cudaLaunchKernelEx(&cfg, fa_splitkv_combine<128>, (const float*)o_part,
+                                   (const float*)lse_part, o, a.lse, (int64_t)rows, a.splits,
+                                   (const uint32_t*)err);
         else
-            fa_splitkv_combine<64><<<cgrid, cblock, 0, s>>>(o_part, lse_part, o, a.lse, rows, a.splits,
-                                                              err);
-        if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+            e = cudaLaunchKernelEx(&cfg, fa_splitkv_combine<64>, (const float*)o_part,
+                                   (const float*)lse_part, o, a.lse, (int64_t)rows, a.splits,
+                                   (const uint32_t*)err);
+        if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
     }
     return FA_OK;
 }
@@ -596,19 +616,25 @@ FA_EXPORT int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, 
         sms = 148;
     int G = 1, nq_blk = fa::kTile;
     fa::tile_shape(H, H_kv, Nq, true, &G, &nq_blk);
-    (void)d;   // one query tile per unit at every d
     const int64_t n_rb = ((int64_t)Nq + nq_blk - 1) / nq_blk;
     const int64_t base = (int64_t)B * (H / G) * n_rb;
     const int64_t key_tiles = ((int64_t)Nk + fa::kTile - 1) / fa::kTile;
     // Each unit pays a fixed cost (its Q tile, the first scores, the epilogue and
     // the partials the merge reads back), and a second wave of units leaves most
     // SMs idle for its last part, so the units are kept to one wave: as many
-    // ranges as fit base * ranges <= SMs, each at least four key tiles long; a
-    // workload with at least as many units as SMs takes one range. (Measured on
-    // one head group of 131072 keys: 18 ranges, 144 units, 5493 GB/s; 16 ranges,
-    // 128 units, 5069; 24 ranges, two waves, 3663.)
+    // ranges as fit base * ranges <= the cap, each at least four key tiles long;
+    // a workload with at least as many units as the cap takes one range. The cap
+    // is the SM count for the general kernel (measured on one head group of
+    // 131072 keys: 18 ranges, 144 units, 5493 GB/s; 16 ranges, 128 units, 5069;
+    // 24 ranges, two waves, 3663). The transposed decoding tile (d = 128, G * Nq
+    // <= 8 columns) streams K and V at the HBM rate and ran fastest with 128
+    // units in flight on every shape measured (1, 2 or 4 sequences x 8 K/V heads,
+    // one query row: 6007, 6116, 6186 GB/s at 128 units against 5655 and 5692
+    // at 144), so its cap is 128.
+    const bool dec = d == 128 && G == H / H_kv && nq_blk == Nq && (int64_t)G * Nq <= fa::kDecLive;
+    const int64_t cap = dec ? std::min<int64_t>(sms, 128) : sms;
     const int64_t s_max = std::min<int64_t>(fa::kMaxSplits, std::max<int64_t>(1, key_tiles / 4));
-    const int64_t sp = base >= sms ? 1 : sms / base;
+    const int64_t sp = base >= cap ? 1 : cap / base;
     return (int)std::max<int64_t>(1, std::min<int64_t>(sp, s_max));
 }
 

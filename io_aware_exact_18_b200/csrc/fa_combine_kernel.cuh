@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "sm100_ptx.cuh"
+
 namespace fa {
 
 constexpr int kCombineWarps = 8;   // rows per 256-thread block
@@ -26,6 +28,9 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
                        int splits, const uint32_t* dev_err) {
     constexpr int kPer = D / 32;   // columns per lane: 2, 4 or 8
     constexpr float kLog2e = 1.4426950408889634f;
+    // Launched as a programmatic dependent of the decoding kernel it may start
+    // early: nothing is read before that kernel has completed.
+    pdl_wait_prerequisites();
     const int64_t row = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;

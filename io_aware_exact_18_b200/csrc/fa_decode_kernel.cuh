@@ -221,6 +221,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // The split-KV merge queued behind this grid may be scheduled once every
+    // CTA has started (it waits for this grid's completion before any read):
+    // its launch overlaps this grid's tail instead of following it.
+    pdl_launch_dependents();
     const uint32_t tmem = bars->tmem_base;
     const bool skip = bars->skip != 0;
     const Watchdog wd{&bars->abort, p.dev_err, p.watchdog_ns};

@@ -189,6 +189,20 @@ __device__ __forceinline__ int clc_decode(const void* resp) {
     return ok ? (int)x : -1;
 }
 
+// Programmatic dependent launch: let the grid queued after this one on the
+// stream (launched with the programmatic-serialization attribute) start once
+// every CTA of this grid has executed this or exited...
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ...and, in that dependent grid, wait until the grid before it has completed
+// and its memory is visible (returns at once for a launch without that
+// attribute).
+__device__ __forceinline__ void pdl_wait_prerequisites() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Order this thread's generic-proxy shared-memory accesses before later
 // async-proxy ones (e.g. reusing a response buffer).
 __device__ __forceinline__ void fence_proxy_async_smem() {
