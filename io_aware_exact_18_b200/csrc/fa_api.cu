@@ -72,10 +72,10 @@ bool set_smem() {
                                 Cfg<D, QT, E>::kSmemBytes) == cudaSuccess;
 }
 
-template <int D>
+template <int D, int E>
 bool set_decode_smem() {
-    return cudaFuncSetAttribute(fa_decode_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                DecCfg<D>::kSmemBytes) == cudaSuccess;
+    return cudaFuncSetAttribute(fa_decode_sm100<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                DecCfg<D, E>::kSmemBytes) == cudaSuccess;
 }
 
 std::mutex g_mutex;
@@ -117,7 +117,7 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
                             set_smem<128, 1, true>() && set_smem<256, 1, true>() &&
                             set_smem<128, 2, false, 1>() && set_smem<256, 1, false, 1>() &&
                             set_smem<128, 1, true, 1>() && set_smem<256, 1, true, 1>() &&
-                            set_decode_smem<128>() &&
+                            set_decode_smem<128, 2>() && set_decode_smem<128, 1>() &&
                             set_bwd_smem<64>() &&
                             set_bwd_smem<128>();
             if (!ok) return FA_ERR_LAUNCH;
@@ -381,13 +381,15 @@ int fwd_impl(const FwdCall& a, void* stream) {
 
     const dim3 grid((unsigned)(BHB * n_units)), block(kThreads);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // Decoding shapes (bf16, d = 128, a K/V group's query heads times the query
-    // rows within kDecLive columns: one row block per group) take the
-    // transposed tile; the unit grid is the same (head group, range) set.
-    const bool dec = E == 2 && d == 128 && pl.general && Nq == nq_blk &&
-                     (int64_t)G * Nq <= kDecLive && G == H / H_kv;
-    if (dec) {
-        fa_decode_sm100<128><<<grid, dim3(kDecThreads), DecCfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
+    // Decoding shapes (d = 128, a K/V group's query heads times the query rows
+    // within kDecLive columns: one row block per group) take the transposed
+    // tile; the unit grid is the same (head group, range) set.
+    const bool dec = d == 128 && pl.general && Nq == nq_blk && (int64_t)G * Nq <= kDecLive &&
+                     G == H / H_kv;
+    if (dec && E == 2) {
+        fa_decode_sm100<128, 2><<<grid, dim3(kDecThreads), DecCfg<128, 2>::kSmemBytes, s>>>(mq, mk, mv, p);
+    } else if (dec) {
+        fa_decode_sm100<128, 1><<<grid, dim3(kDecThreads), DecCfg<128, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
     } else if (E == 1) {
         if (pl.general && d == 256)
             fa_fwd_sm100<256, 1, true, 1><<<grid, block, Cfg<256, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);

@@ -65,30 +65,34 @@ constexpr int kDecThreads = 320;
 constexpr int kDecTmaWarp = 8;
 constexpr int kDecMmaWarp = 9;
 
-template <int D>
+// E: bytes per element of Q, K, V and P (2: bf16; 1: e4m3 with kind::f8f6f4
+// products, P rounded to e4m3).
+template <int D, int E>
 struct DecCfg {
     static_assert(D == 128, "the transposed decode tile is built for d = 128");
+    static_assert(E == 1 || E == 2, "bf16 or e4m3");
     static_assert(kDecLive <= kDecCols, "live columns within the product's N");
-    static constexpr int kBlocks = D / 64;                   // 128-byte column blocks per row
+    static constexpr int kBlocks = D * E / 128;              // 128-byte column blocks per row
+    static constexpr int kBlockElems = 128 / E;
     static constexpr int kBlockBytes = kTile * 128;          // 16 KB: one block of a K/V tile
-    static constexpr int kTileBytes = kTile * D * 2;         // 32 KB
+    static constexpr int kTileBytes = kTile * D * E;         // 32 KB (bf16), 16 KB (e4m3)
     static constexpr int kColBlockBytes = kDecCols * 128;    // 2 KB: one block of a 16-row operand
-    static constexpr int kQBytes = kBlocks * kColBlockBytes; // 4 KB
-    static constexpr int kPBytes = (kTile / 64) * kColBlockBytes;   // 4 KB: 16 x 128 keys
-    static constexpr int kSlots = 6;                         // K/V ring depth
+    static constexpr int kQBytes = kBlocks * kColBlockBytes;
+    static constexpr int kPBytes = (kTile * E / 128) * kColBlockBytes;   // 16 x 128 keys
+    static constexpr int kSlots = E == 2 ? 6 : 12;           // K/V ring depth
     static constexpr int kSmemTiles = kQBytes + 2 * kPBytes + kSlots * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 4096 /*barriers*/;
     static constexpr uint32_t kTmemCols = 64;
     static constexpr uint32_t col_s(int w) { return (uint32_t)(w * kDecCols); }
     static constexpr uint32_t col_o(int w) { return (uint32_t)((2 + w) * kDecCols); }
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-    static_assert(kSlots <= 8, "K/V ring barriers");
+    static_assert(kSlots <= 12, "K/V ring barriers");
 };
 
 struct DecBarriers {
     uint64_t q_full;
-    uint64_t kv_full[8];
-    uint64_t kv_empty[8];
+    uint64_t kv_full[12];
+    uint64_t kv_empty[12];
     // per warpgroup w (= key-tile parity)
     uint64_t s_full[2];       // S^T of a key tile is in TMEM (MMA commit)
     uint64_t s_free[2];       // its 128 threads have read it (128 arrivals)
@@ -136,20 +140,23 @@ __device__ __forceinline__ float warp_reduce_scatter8(const float (&v)[kDecLive]
     return op(w1, __shfl_xor_sync(0xffffffffu, w1, 1));
 }
 
-// Byte offset of element (row n, column k) of a K-major operand of 16 rows in
-// the 128-byte swizzled layout: 64-column blocks of 2 KB, rows of 128 bytes,
-// the 16-byte chunk index XOR-ed with the row index mod 8.
+// Byte offset of element (row n, column k) of a K-major operand of 16 rows of
+// E-byte elements in the 128-byte swizzled layout: 128-byte column blocks of
+// 2 KB, rows of 128 bytes, the 16-byte chunk index XOR-ed with the row index
+// mod 8.
+template <int E>
 __device__ __forceinline__ uint32_t kmajor16_offset(int n, int k) {
-    return (uint32_t)((k >> 6) * (kDecCols * 128) + n * 128 +
-                      ((((k & 63) >> 3) ^ (n & 7)) << 4) + (k & 7) * 2);
+    const int kb = k * E;
+    return (uint32_t)((kb >> 7) * (kDecCols * 128) + n * 128 +
+                      ((((kb & 127) >> 4) ^ (n & 7)) << 4) + (kb & 15));
 }
 
-template <int D>
+template <int D, int E>
 __global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_sm100(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = DecCfg<D>;
+    using C = DecCfg<D, E>;
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             bool ok = true;
             mbar_arrive_expect_tx(&bars->q_full, (uint32_t)(C::kBlocks * cols * 128));
             for (int blk = 0; blk < C::kBlocks; ++blk)
-                tma_load_3d(&tm_q, &bars->q_full, sQ + blk * C::kColBlockBytes, blk * 64, 0,
+                tma_load_3d(&tm_q, &bars->q_full, sQ + blk * C::kColBlockBytes, blk * C::kBlockElems, 0,
                             b * p.H + h0);
             // Loads in the order the MMAs consume them: K0 | K1 V0 | K2 V1 | ... | V(n-1).
             const int loads = 2 * n;
@@ -263,7 +270,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
                 for (int blk = 0; blk < C::kBlocks; ++blk)
                     tma_load_3d_hint(is_v ? &tm_v : &tm_k, &bars->kv_full[slot],
-                                     dst + blk * C::kBlockBytes, blk * 64, (kt0 + tile) * kTile,
+                                     dst + blk * C::kBlockBytes, blk * C::kBlockElems, (kt0 + tile) * kTile,
                                      bkv, pol_kv);
                 ++issued;
             }
@@ -276,8 +283,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     } else if (warp == kDecMmaWarp) {
         // ====================================================== MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, kDecCols, 0, 0);   // K . Q^T
-            constexpr uint32_t idesc_o = idesc_bf16_f32(128, kDecCols, 1, 0);   // V^T . P^T
+            constexpr uint32_t idesc_s = E == 2 ? idesc_bf16_f32(128, kDecCols, 0, 0)   // K . Q^T
+                                                : idesc_e4m3_f32(128, kDecCols, 0, 0);
+            constexpr uint32_t idesc_o = E == 2 ? idesc_bf16_f32(128, kDecCols, 1, 0)   // V^T . P^T
+                                                : idesc_e4m3_f32(128, kDecCols, 1, 0);
+            auto mma = [&](uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+                if constexpr (E == 2) umma_ss(d_tmem, a, b, idesc, acc);
+                else umma_ss_f8(d_tmem, a, b, idesc, acc);
+            };
             const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(smem_u32(sKV), 16, 1024);          // K-major
             const uint64_t dv0 = smem_desc_sw128(smem_u32(sKV), C::kBlockBytes, 1024); // MN-major
@@ -299,10 +312,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     tc_fence_after();
                     const uint64_t a = dk0 + (uint64_t)slot * kTileStep;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
+                    for (int kk = 0; kk < D * E / 32; ++kk) {       // 32-byte K-steps
                         const uint64_t oa = (uint64_t)(((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4);
                         const uint64_t ob = (uint64_t)(((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4);
-                        umma_ss(tmem + C::col_s(w), a + oa, dq + ob, idesc_s, kk > 0 ? 1u : 0u);
+                        mma(tmem + C::col_s(w), a + oa, dq + ob, idesc_s, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(&bars->s_full[w]);
                     umma_commit(&bars->kv_empty[slot]);
@@ -319,11 +332,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     const uint64_t a = dv0 + (uint64_t)slot * kTileStep;
                     const uint64_t bp = dp0 + (uint64_t)w * kPStep;
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint64_t oa = (uint64_t)((kk * 16 * 128) >> 4);
+                    for (int kk = 0; kk < kTile * E / 32; ++kk) {   // 32 / E keys per K-step
+                        const uint64_t oa = (uint64_t)((kk * (32 / E) * 128) >> 4);
                         const uint64_t ob = (uint64_t)(((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4);
-                        umma_ss(tmem + C::col_o(w), a + oa, bp + ob, idesc_o,
-                                (jj > 1 || kk > 0) ? 1u : 0u);
+                        mma(tmem + C::col_o(w), a + oa, bp + ob, idesc_o, (jj > 1 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(&bars->pv_done[w]);
                     umma_commit(&bars->p_free[w]);
@@ -393,7 +405,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             for (int q = 0; q < kDecLive; ++q) {
                 const float tmax = tile_max(q);
                 if (m_ref[q] == -INFINITY) m_ref[q] = tmax;
-                else if ((tmax - m_ref[q]) * c > 64.f) rescale = true;
+                else if ((tmax - m_ref[q]) * c > rescale_log2<E>()) rescale = true;
             }
             if (rescale) {   // uniform in the warpgroup: every thread sees the same maxima
                 // O^T(wg) holds the products of this warpgroup's tiles < j; the
@@ -410,7 +422,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
                 for (int q = 0; q < kDecLive; ++q) {
                     const float tmax = tile_max(q);
-                    if ((tmax - m_ref[q]) * c > 64.f) {
+                    if ((tmax - m_ref[q]) * c > rescale_log2<E>()) {
                         const float alpha = fast_exp2((m_ref[q] - tmax) * c);
                         m_ref[q] = tmax;
                         l[q] *= alpha;
@@ -422,21 +434,38 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 tmem_wait_st();
             }
 
-            // probabilities of this key, rounded to bf16 into the warpgroup's P^T
+            // probabilities of this key, rounded to bf16 (e4m3) into the warpgroup's P^T
             if (jo >= 1) {   // P.V(j - 2) has read the buffer (complete, as above)
                 ok = mbar_wait(&bars->p_free[wg], (uint32_t)(jo - 1) & 1u, wd);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
             }
             uint8_t* pbuf = sP + wg * C::kPBytes;
+            float pv[kDecLive];
 #pragma unroll
             for (int q = 0; q < kDecLive; ++q) {
                 const float mc = (m_ref[q] == -INFINITY) ? 0.f : m_ref[q] * c;
-                const float pv = fast_exp2(fmaf(s[q], c, -mc));
-                const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
-                l[q] += pv;
-                lr[q] += __bfloat162float(pb);
-                *reinterpret_cast<__nv_bfloat16*>(pbuf + kmajor16_offset(q, t)) = pb;
+                pv[q] = fast_exp2(fmaf(s[q], c, -mc));
+                l[q] += pv[q];
+            }
+            if constexpr (E == 2) {
+#pragma unroll
+                for (int q = 0; q < kDecLive; ++q) {
+                    const __nv_bfloat16 pb = __float2bfloat16_rn(pv[q]);
+                    lr[q] += __bfloat162float(pb);
+                    *reinterpret_cast<__nv_bfloat16*>(pbuf + kmajor16_offset<E>(q, t)) = pb;
+                }
+            } else {
+                // e4m3 P: O is divided by the exact sum, as in the e4m3 forward
+#pragma unroll
+                for (int q4 = 0; q4 < kDecLive; q4 += 4) {
+                    const uint32_t w4 = pack_e4m3x4(pv[q4], pv[q4 + 1], pv[q4 + 2], pv[q4 + 3]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pbuf[kmajor16_offset<E>(q4 + e, t)] = (uint8_t)(w4 >> (8 * e));
+                }
+#pragma unroll
+                for (int q = 0; q < kDecLive; ++q) lr[q] += pv[q];
             }
             fence_proxy_async_smem();    // the P.V product reads P^T through the async proxy
             tc_fence_before();

@@ -147,3 +147,39 @@ def test_fp8_splitkv_key_padding(fa, d):
     compare_fp8(o, lse, o_ref, lse_ref, vmax, f"kv_len padding d{d}")
     assert np.all(o[0] == 0.0) and np.all(np.isneginf(lse[0]))
 
+
+
+@pytest.mark.parametrize("H,H_kv,Nq,causal", [
+    (8, 2, 1, True),      # 4 heads per K/V head: the transposed decoding tile
+    (8, 1, 1, False),     # 8 columns, the tile's limit
+    (4, 4, 2, True),      # one head per group, 2 rows
+    (2, 1, 4, False),     # 8 columns from 2 heads x 4 rows
+    (1, 1, 9, True),      # 9 columns: the general kernel
+])
+def test_fp8_decoding_tile(fa, H, H_kv, Nq, causal):
+    """e4m3 decoding through fa_fwd_splitkv_fp8 at d = 128, on both sides of the
+    transposed tile's 8-column limit, at the default and two fixed range counts."""
+    for splits in (None, 1, 3):
+        check_fp8(fa, 2, H, H_kv, Nq, causal, seed=6800 + 7 * H + Nq, d=128, Nk=3000,
+                  splits=splits)
+
+
+def test_fp8_decoding_reference_moves_every_tile(fa):
+    """e4m3 scores that grow by more than 8 log2 units from one key tile to the
+    next (q = 32 and every key of tile t equal to 2t along one axis, exact in
+    e4m3), so every column's reference maximum moves at every tile."""
+    B, H, H_kv, Nq, Nk, d = 1, 4, 1, 1, 11 * 128, 128
+    q = torch.zeros(B, H, Nq, d)
+    q[..., 0] = 32.0
+    k = torch.zeros(B, H_kv, Nk, d)
+    k[..., 0] = 2.0 * (torch.arange(Nk) // 128).float()
+    g = torch.Generator().manual_seed(4)
+    v = torch.randn(B, H_kv, Nk, d, generator=g)
+    q8, k8, v8 = (x.to(torch.float8_e4m3fn) for x in (q, k, v))
+    assert 32 * 2 / math.sqrt(d) * math.log2(math.e) > 8
+    sc = (1.0, 1.0, 1.0)
+    for splits in (1, 3):
+        o, lse = run_fp8(fa, q8, k8, v8, sc, False, cache=True, splits=splits)
+        o_ref, lse_ref = ofp8.attention_fp8(q8, k8, v8, *sc, 1.0 / math.sqrt(d))
+        vmax = float(np.abs(ofp8.decode_e4m3(v8.view(torch.uint8).numpy())).max())
+        compare_fp8(o, lse, o_ref, lse_ref, vmax, f"e4m3 moving reference splits={splits}")
