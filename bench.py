@@ -324,6 +324,16 @@ def reference_arm(args, w):
 
 
 # ----------------------------------------------------------------- GPU arm
+def decode_kernel_name(w, splits: int) -> str:
+    """The kernels a split-KV call of decode workload w launches: the
+    transposed decoding tile when the query heads of a K/V group times the
+    query rows fit its 8 columns at d = 128, else the general kernel; then the
+    merge when there is more than one key range."""
+    tile = (w.d == 128 and (w.H // w.H_kv) * w.Nq <= 8)
+    name = "fa_decode_sm100<128,bf16>" if tile else f"fa_fwd_sm100<{w.d},1,general>"
+    return name + (f" + fa_splitkv_combine<{w.d}>" if splits > 1 else "")
+
+
 def max_over_ranks(x: float, world: int) -> float:
     if world <= 1:
         return x
@@ -713,7 +723,7 @@ def decode_arm(args, w):
                 "peak_source": f"{peak_src} copy bandwidth",
                 "algorithmic_bytes": float(nbytes),
                 "timed": "whole step: attention kernel over all key ranges + merge kernel",
-                "kernel": f"fa_fwd_sm100<{w.d},1,general> + fa_splitkv_combine<{w.d}>"}
+                "kernel": decode_kernel_name(w, splits)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle

@@ -46,15 +46,19 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
         return;
     }
 
-    // Pass 1: the largest lse_s (lane l reads splits l, l + 32, ...).
-    float m = -INFINITY;
-    for (int s = lane; s < splits; s += 32) m = fmaxf(m, lse_part[(int64_t)s * rows + row]);
+    // Pass 1: the largest lse_s (lane l reads splits l, l + 32, ...; the first
+    // is kept for pass 2).
+    const float ls0 = (lane < splits) ? lse_part[(int64_t)lane * rows + row] : -INFINITY;
+    float m = ls0;
+    for (int s = lane + 32; s < splits; s += 32) m = fmaxf(m, lse_part[(int64_t)s * rows + row]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
 
     // Pass 2: weights exp(lse_s - m), one split per lane, broadcast by shuffle;
     // the O_s rows are loaded unconditionally (an empty range wrote O_s = 0 and
-    // has weight 0), so the loads of consecutive splits overlap.
+    // has weight 0) as 16-byte vectors, eight splits per unrolled step, so a
+    // warp has that many rows' loads in flight (the merge is latency-bound: a
+    // handful of rows per SM).
     float acc[kPer];
 #pragma unroll
     for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
@@ -62,20 +66,29 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
     if (m != -INFINITY) {
         for (int base = 0; base < splits; base += 32) {
             const int sl = base + lane;
-            const float ls = (sl < splits) ? lse_part[(int64_t)sl * rows + row] : -INFINITY;
+            const float ls = (base == 0) ? ls0
+                             : (sl < splits) ? lse_part[(int64_t)sl * rows + row] : -INFINITY;
             const float wl = (ls == -INFINITY) ? 0.f : exp2f((ls - m) * kLog2e);
             wsum += wl;
             const int cnt = min(32, splits - base);
             const float* src = o_part + ((int64_t)base * rows + row) * D + lane * kPer;
-#pragma unroll 4
+#pragma unroll 8
             for (int j = 0; j < cnt; ++j) {
                 const float w = __shfl_sync(0xffffffffu, wl, j);
                 const float* r = src + (int64_t)j * rows * D;
+                if constexpr (kPer % 4 == 0) {
 #pragma unroll
-                for (int c = 0; c < kPer; c += 2) {
-                    const float2 x = *reinterpret_cast<const float2*>(r + c);
-                    acc[c] = fmaf(w, x.x, acc[c]);
-                    acc[c + 1] = fmaf(w, x.y, acc[c + 1]);
+                    for (int c = 0; c < kPer; c += 4) {
+                        const float4 x = *reinterpret_cast<const float4*>(r + c);
+                        acc[c] = fmaf(w, x.x, acc[c]);
+                        acc[c + 1] = fmaf(w, x.y, acc[c + 1]);
+                        acc[c + 2] = fmaf(w, x.z, acc[c + 2]);
+                        acc[c + 3] = fmaf(w, x.w, acc[c + 3]);
+                    }
+                } else {
+                    const float2 x = *reinterpret_cast<const float2*>(r);
+                    acc[0] = fmaf(w, x.x, acc[0]);
+                    acc[1] = fmaf(w, x.y, acc[1]);
                 }
             }
         }

@@ -141,3 +141,18 @@ def test_time_steps_flushes_before_each_step_and_times_only_the_step():
     ms = bench.time_steps(fake_torch, _FakeStream(log), step, 4, None)
     assert [e[0] for e in log] == ["record"] + ["step"] * 4 + ["record", "sync"]
     assert ms == pytest.approx(2.0 / 4)
+
+
+def test_decode_kernel_name_follows_the_dispatch_rule():
+    """The decode line names the transposed tile exactly where the library
+    takes it (d = 128, query heads per K/V head x query rows <= 8), and the
+    merge only when there is more than one key range."""
+    import workloads
+    w1, w2 = workloads.DECODE_WORKLOADS[0], workloads.DECODE_WORKLOADS[1]
+    assert bench.decode_kernel_name(w1, 1) == "fa_decode_sm100<128,bf16>"
+    assert bench.decode_kernel_name(w2, 16) == \
+        "fa_decode_sm100<128,bf16> + fa_splitkv_combine<128>"
+    wide = workloads.DecodeWorkload("wide", 1, 32, 2, 1, 4096, 128)   # 16 heads per K/V head
+    assert bench.decode_kernel_name(wide, 4).startswith("fa_fwd_sm100<128,1,general>")
+    d64 = workloads.DecodeWorkload("d64", 1, 32, 8, 1, 4096, 64)
+    assert bench.decode_kernel_name(d64, 1) == "fa_fwd_sm100<64,1,general>"
