@@ -156,9 +156,8 @@ int fa_splitkv_default_splits(int B, int H, int H_kv, int Nq, int Nk, int d);
  * section "FlashAttention-3"): both tile products run on the tensor cores in
  * e4m3 with fp32 accumulation, and the probabilities P are rounded to e4m3
  * (relative error up to 2^-4) before the P.V product, so O carries that
- * error; lse does not (scores are exact products of e4m3 values). d must be
- * 128 or 256 (d = 64: FA_ERR_UNSUPPORTED); causal, kv_len, H_kv, errors as in
- * fa_fwd_gqa.
+ * error; lse does not (scores are exact products of e4m3 values). d is 64,
+ * 128 or 256; causal, kv_len, H_kv, errors as in fa_fwd_gqa.
  */
 int fa_fwd_fp8(const void *q, const void *k, const void *v, float q_descale, float k_descale,
                float v_descale, void *o, float *lse, int B, int H, int H_kv, int N, int d,
@@ -169,8 +168,8 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, float q_descale, flo
  * [B, H_kv, Nk, d] and their descales as in fa_fwd_fp8 (same precision
  * statement). O bf16 [B, H, Nq, d], lse fp32 [B, H, Nq]; the partials in
  * `workspace` are fp32, sized by fa_splitkv_workspace_bytes as for bf16
- * inputs. d must be 128 or 256 (d = 64: FA_ERR_UNSUPPORTED); every other
- * argument and error as in fa_fwd_splitkv.
+ * inputs. d is 64, 128 or 256; every other argument and error as in
+ * fa_fwd_splitkv.
  */
 int fa_fwd_splitkv_fp8(const void *q, const void *k, const void *v, float q_descale,
                        float k_descale, float v_descale, void *o, float *lse, int B, int H,

@@ -117,6 +117,7 @@ int prepare_device(int* dev_out, uint32_t** err_out) {
                             set_smem<128, 1, true>() && set_smem<256, 1, true>() &&
                             set_smem<128, 2, false, 1>() && set_smem<256, 1, false, 1>() &&
                             set_smem<128, 1, true, 1>() && set_smem<256, 1, true, 1>() &&
+                            set_smem<64, 2, false, 1>() && set_smem<64, 1, true, 1>() &&
                             set_decode_smem<128, 2>() && set_decode_smem<128, 1>() &&
                             set_bwd_smem<64>() &&
                             set_bwd_smem<128>();
@@ -144,12 +145,17 @@ int encode_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_
     if (!enc) return FA_ERR_LAUNCH;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)d * elem, (cuuint64_t)N * (cuuint64_t)d * elem};
-    cuuint32_t box[3] = {(cuuint32_t)(128 / elem), (cuuint32_t)box_rows, (cuuint32_t)box_planes};
+    // one column block of a tile per box: 128-byte rows with the 128-byte
+    // swizzle, or whole 64-byte rows (e4m3 at d = 64) with the 64-byte swizzle
+    const int row_bytes = std::min(128, d * elem);
+    cuuint32_t box[3] = {(cuuint32_t)(row_bytes / elem), (cuuint32_t)box_rows,
+                         (cuuint32_t)box_planes};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                      3, const_cast<void*>(ptr), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
 }
@@ -268,7 +274,6 @@ int fwd_check(const FwdCall& a, FwdPlan* pl) {
     if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     const int E = a.elem;
     if (E == 1) {
-        if (d == 64) return FA_ERR_UNSUPPORTED;   // e4m3: d = 128 or 256
         for (float x : {a.q_descale, a.k_descale, a.v_descale})
             if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
     }
@@ -393,12 +398,16 @@ int fwd_impl(const FwdCall& a, void* stream) {
     } else if (E == 1) {
         if (pl.general && d == 256)
             fa_fwd_sm100<256, 1, true, 1><<<grid, block, Cfg<256, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
-        else if (pl.general)
+        else if (pl.general && d == 128)
             fa_fwd_sm100<128, 1, true, 1><<<grid, block, Cfg<128, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else if (pl.general)
+            fa_fwd_sm100<64, 1, true, 1><<<grid, block, Cfg<64, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
         else if (d == 256)
             fa_fwd_sm100<256, 1, false, 1><<<grid, block, Cfg<256, 1, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
-        else
+        else if (d == 128)
             fa_fwd_sm100<128, 2, false, 1><<<grid, block, Cfg<128, 2, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
+        else
+            fa_fwd_sm100<64, 2, false, 1><<<grid, block, Cfg<64, 2, 1>::kSmemBytes, s>>>(mq, mk, mv, p);
     } else if (pl.general) {
         if (d == 256)
             fa_fwd_sm100<256, 1, true><<<grid, block, Cfg<256, 1>::kSmemBytes, s>>>(mq, mk, mv, p);

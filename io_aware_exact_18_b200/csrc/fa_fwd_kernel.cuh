@@ -107,20 +107,26 @@ constexpr float kLn2 = 0.69314718055994530942f;
 // current ones. d = 256 needs it (O alone takes 256 TMEM columns); the
 // split-KV kernel uses it at every d, since a short query block gives the
 // second tile of a pair nothing to do.
-// E is the element size of Q, K and V: 2 (bf16) or 1 (e4m3, d = 128 or 256:
-// a 64-byte row at d = 64 would need another swizzle layout).
+// E is the element size of Q, K and V: 2 (bf16) or 1 (e4m3). Tiles are stored
+// in column blocks of swizzle rows: 128-byte rows with the 128-byte swizzle,
+// or, when a whole row is 64 bytes (e4m3 at d = 64), 64-byte rows with the
+// 64-byte swizzle.
 template <int D, int QT, int E = 2>
 struct Cfg {
     static_assert(D == 64 || D == 128 || D == 256, "head dim 64, 128 or 256");
     static_assert(QT == 1 || (QT == 2 && D <= 128), "two query tiles need d <= 128");
-    static_assert(E == 2 || (E == 1 && D >= 128), "e4m3 inputs need d = 128 or 256");
+    static_assert(E == 1 || E == 2, "bf16 or e4m3");
     static constexpr int kQT = QT;                        // query tiles per unit
-    static constexpr int kBlocks = D * E / 128;           // 128-byte column blocks per row
-    static constexpr int kBlockElems = 128 / E;           // columns of one block
-    static constexpr int kBlockBytes = kTile * 128;       // 16 KB
+    static constexpr int kRowBytes = D * E < 128 ? D * E : 128;   // bytes of one swizzle row
+    static constexpr int kSwizzle = kRowBytes == 128 ? 2 : 4;     // descriptor code: 128- / 64-byte
+    static constexpr int kBlocks = D * E / kRowBytes;     // column blocks per row
+    static constexpr int kBlockElems = kRowBytes / E;     // columns of one block
+    static constexpr int kBlockBytes = kTile * kRowBytes; // 16 KB (8 KB with 64-byte rows)
+    static constexpr int kAtomBytes = 8 * kRowBytes;      // 8 rows: the swizzle pattern's period
+    static constexpr int kStepsPerBlock = kRowBytes / 32; // 32-byte K-steps in one row
     static constexpr int kTileBytes = kTile * D * E;      // one Q/K/V tile
     static constexpr int kSlots =                         // K/V ring depth
-        (D * E == 256) ? (QT == 2 ? 4 : 5) : (D * E == 512) ? 2 : 8;
+        (D * E == 256) ? (QT == 2 ? 4 : 5) : (D * E == 512) ? 2 : 8;   // 8 at 64 or 128 bytes
     static constexpr int kSmemTiles = (kQT + kSlots) * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 4096 /*barriers*/;
     static constexpr uint32_t kTmemCols = 512;
@@ -476,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint64_t pol_kv = policy_evict_last();
             const uint64_t pol_q = policy_evict_first();
-            const uint32_t q_bytes = (uint32_t)(C::kBlocks * sh.G * sh.nq_blk * 128);
+            const uint32_t q_bytes = (uint32_t)(C::kBlocks * sh.G * sh.nq_blk * C::kRowBytes);
             int id = skip ? -1 : (int)blockIdx.x;
             int L = 0;                 // K/V loads issued (K_j and V_j of every unit, in order)
             int k = 0;                 // units published
@@ -588,9 +594,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr int kStepRows = 32 / E;                  // keys per 32-byte K-step
             // Descriptors are built once; a tile's start address is added in
             // 16-byte units to the low field (addresses stay below 256 KB).
-            const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ[0]), 16, 1024);
-            const uint64_t dk0 = smem_desc_sw128(smem_u32(sKV), 16, 1024);            // K-major
-            const uint64_t dv0 = smem_desc_sw128(smem_u32(sKV), C::kBlockBytes, 1024); // MN-major
+            const uint64_t dq0 = smem_desc(smem_u32(sQ[0]), 16, C::kAtomBytes, C::kSwizzle);
+            const uint64_t dk0 = smem_desc(smem_u32(sKV), 16, C::kAtomBytes, C::kSwizzle);  // K-major
+            const uint64_t dv0 =                                                              // MN-major
+                smem_desc(smem_u32(sKV), C::kBlockBytes, C::kAtomBytes, C::kSwizzle);
             constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
             // S buffer sb = Q tile t . K tile in `slot`
             auto issue_qk = [&](int t, int sb, int slot) {
@@ -599,7 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D * E / 32; ++kk) {      // 32-byte K-steps
                     const uint64_t off =
-                        (uint64_t)(((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4);
+                        (uint64_t)(((kk / C::kStepsPerBlock) * C::kBlockBytes +
+                                    (kk % C::kStepsPerBlock) * 32) >> 4);
                     if constexpr (E == 2)
                         umma_ss(tmem + C::col_s(sb), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
                     else
@@ -618,8 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < kTile / kStepRows; ++kk) {
 #pragma unroll
                     for (int h = 0; h < kPvHalves; ++h) {
-                        const uint64_t bk = b + (uint64_t)((kk * kStepRows * 128 +
-                                                            h * (kPvN * E / 128) * C::kBlockBytes) >> 4);
+                        const uint64_t bk = b + (uint64_t)((kk * kStepRows * C::kRowBytes +
+                                                            h * (kPvN * E / C::kRowBytes) * C::kBlockBytes) >> 4);
                         if constexpr (E == 2)
                             umma_ts(tmem + C::col_o(t) + (uint32_t)(h * kPvN),
                                     tP + (uint32_t)(kk * 8), bk, idesc_pv,

@@ -369,16 +369,22 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 // Shared-memory matrix descriptor (tcgen05 format): start address >> 4 in
 // bits [0,14), leading-dimension byte offset >> 4 in [16,30), stride-dimension
 // byte offset >> 4 in [32,46), version 1 in [46,48), swizzle mode in [61,64)
-// (2 = 128-byte swizzle). Base offset 0: tiles are 1024-byte aligned.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
+// (2 = 128-byte swizzle, 4 = 64-byte swizzle). Base offset 0: tiles are
+// 1024-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint32_t swizzle) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
     d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
+    d |= (uint64_t)(swizzle & 7u) << 61;
     return d;
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+    return smem_desc(saddr, lbo_bytes, sbo_bytes, 2u);
 }
 
 // Instruction descriptor for kind::f16: fp32 accumulator (bits [4,6) = 1),

@@ -221,8 +221,8 @@ def test_bwd_workspace_bytes(lib):
 
 # ---------------------------------------------------------------- e4m3 forward
 @pytest.mark.parametrize("over,status", [
-    (dict(d=64), fa.FA_ERR_UNSUPPORTED),
     (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=512), fa.FA_ERR_UNSUPPORTED),
     (dict(qs=0.0), fa.FA_ERR_INVALID_ARG),
     (dict(ks=-1.0), fa.FA_ERR_INVALID_ARG),
     (dict(vs=float("inf")), fa.FA_ERR_INVALID_ARG),
@@ -243,7 +243,7 @@ def test_fp8_argument_errors_are_synchronous(lib, over, status):
 
 
 @pytest.mark.parametrize("over,status", [
-    (dict(d=64), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
     (dict(qs=0.0), fa.FA_ERR_INVALID_ARG),
     (dict(vs=float("nan")), fa.FA_ERR_INVALID_ARG),
     (dict(Nq=513), fa.FA_ERR_INVALID_ARG),            # more queries than keys

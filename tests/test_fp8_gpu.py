@@ -1,4 +1,4 @@
-"""GPU parity of the e4m3 forward (fa_fwd_fp8 at d = 128 and 256, and the
+"""GPU parity of the e4m3 forward (fa_fwd_fp8 at d = 64, 128 and 256, and the
 split-KV form fa_fwd_splitkv_fp8) against the fp64 oracle on the dequantized
 inputs (oracle.fp8.attention_fp8).
 
@@ -183,3 +183,20 @@ def test_fp8_decoding_reference_moves_every_tile(fa):
         o_ref, lse_ref = ofp8.attention_fp8(q8, k8, v8, *sc, 1.0 / math.sqrt(d))
         vmax = float(np.abs(ofp8.decode_e4m3(v8.view(torch.uint8).numpy())).max())
         compare_fp8(o, lse, o_ref, lse_ref, vmax, f"e4m3 moving reference splits={splits}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 129, 300, 1024])
+def test_fp8_head_dim_64(fa, N, causal):
+    """d = 64: a row is 64 bytes, stored with the 64-byte swizzle (TMA box and
+    tcgen05 descriptors), two query tiles per unit."""
+    check_fp8(fa, 2, 2, 2, N, causal, seed=6900 + N + causal, d=64)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_head_dim_64_grouped_heads_padding_and_cache(fa, causal):
+    check_fp8(fa, 2, 8, 2, 700, causal, seed=6950 + causal, kv_len_range=(0, 700), d=64)
+    for splits in (None, 1, 3):
+        check_fp8(fa, 2, 8, 2, 5, causal, seed=6960 + causal, d=64, Nk=2000, splits=splits)
+        check_fp8(fa, 1, 4, 4, 200, causal, seed=6970 + causal, d=64, Nk=1000, splits=splits)
+

@@ -140,9 +140,9 @@ N_FP8_MORE = 16
 
 @pytest.mark.parametrize("case", range(N_FP8_MORE))
 def test_random_fp8_d256_and_cache(fa, case):
-    """The e4m3 forward at d = 256 (square) and through the split-KV entry at
-    d = 128 and 256 (fewer query rows than keys, packed heads, key ranges) on
-    seeded random configurations, with the e4m3 bounds."""
+    """The e4m3 forward at d = 64 and 256 (square) and through the split-KV
+    entry at d = 64, 128 and 256 (fewer query rows than keys, packed heads, key
+    ranges) on seeded random configurations, with the e4m3 bounds."""
     from tests.test_fp8_gpu import check_fp8
     rng = np.random.default_rng(4242 + 7919 * case)
     B = int(rng.integers(1, 3))
@@ -150,10 +150,10 @@ def test_random_fp8_d256_and_cache(fa, case):
     H = H_kv * int(rng.choice([1, 2, 4, 8]))
     causal = bool(rng.integers(0, 2))
     if case % 2 == 0:
-        d, N = 256, int(rng.integers(1, 700))
+        d, N = int(rng.choice([64, 256])), int(rng.integers(1, 700))
         Nk, splits = None, None
     else:
-        d = int(rng.choice([128, 256]))
+        d = int(rng.choice([64, 128, 256]))
         Nk = int(rng.integers(1, 1500))
         N = int(rng.integers(1, min(Nk, 200) + 1))
         splits = [None, 1, 2, 5][int(rng.integers(0, 4))]
