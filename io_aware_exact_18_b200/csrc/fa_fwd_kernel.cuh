@@ -15,11 +15,12 @@
 // trims the non-matmul work that "FlashAttention-2 (HI)" section 1 targets.
 // The reference maximum m_ref is set by a row's first key tile and is raised
 // only rarely, so the per-tile rescale of the online softmax becomes an
-// exception. With two query tiles a tile's row maximum is taken before its
-// exponentials and moves m_ref only when it exceeds it by more than 64 in log2
-// units (8 for e4m3 P), after O and l are rescaled; with one query tile each
-// tile is exponentiated against m_ref straight away and the rare tile whose
-// probabilities would sum past 2^64 is redone after the rescale. Both O and l
+// exception. With two query tiles, and for e4m3 inputs, a tile's row maximum
+// is taken before its exponentials and moves m_ref only when it exceeds it by
+// more than 64 in log2 units (8 for e4m3 P), after O and l are rescaled; with
+// one bf16 query tile each tile is exponentiated against m_ref straight away
+// and the rare tile whose probabilities would sum past 2^64 is redone after the
+// rescale. Both O and l
 // share the reference, so the final O / l is unchanged by this choice (the
 // ratio is exact), and every probability stays at most 2^64, far inside the
 // fp32 and bf16 range.
