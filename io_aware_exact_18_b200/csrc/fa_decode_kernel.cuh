@@ -15,8 +15,9 @@
 // (N = 16 is the narrowest tcgen05 product at M = 128; the columns past
 // kDecLive are zero in Q and P^T) so each softmax thread owns one key and 8
 // scores, and the exponential work per key tile drops 16-fold. (Sixteen live
-// columns per thread, in both warpgroups, would not fit the 168 registers a
-// thread of this 320-thread CTA can hold.) The online softmax runs per query column
+// columns per thread would not fit the registers a thread of this CTA can
+// hold: 168 in this 320-thread CTA.) The online softmax runs
+// per query column
 // ("FlashAttention (UR)", section "Online softmax"): a column's reference
 // maximum m_ref is fixed from its first visible key tile and moves only when a
 // later tile's column maximum exceeds it by more than 64 in log2 units, after
@@ -29,26 +30,28 @@
 // probabilities as rounded to bf16 for the P.V product and lse takes the exact
 // sum.
 //
-// Two softmax warpgroups take alternate key tiles (warpgroup w: tiles j with
-// j % 2 == w), each with its own S^T and P^T buffers, O^T accumulator,
-// reference maxima and sums, so the fixed latencies of one tile (TMEM load,
-// shuffles, the maxima exchange, the hand-over) overlap the other's; the
-// epilogue merges the two halves by their log-sum-exp, as the split-KV merge
-// does across ranges.
+// kDecWG = 2 softmax warpgroups take the key tiles in turn (warpgroup w: tiles
+// j with j % kDecWG == w), each with its own S^T and P^T buffers, O^T
+// accumulator, reference maxima and sums, so the fixed latencies of one tile
+// (TMEM load, shuffles, the maxima exchange, the hand-over) overlap the
+// others'; the epilogue merges the parts by their log-sum-exp, as the split-KV
+// merge does across ranges. (Three warpgroups, 448 threads at 128 registers,
+// measured no faster: the tile period is not set by the softmax alone.)
 //
 // One CTA per unit (batch, K/V head group, key range); 320 threads:
-//   warps 0-3  softmax, even key tiles: thread t owns key t of a tile (TMEM
-//              lane t) and, in the epilogue, head-dim index t of O^T
-//   warps 4-7  softmax, odd key tiles
+//   warps 0-3, 4-7  softmax, one warpgroup each: thread t owns key t of a tile
+//              (TMEM lane t) and, in warpgroup 0's epilogue, head-dim index t
+//              of O^T
 //   warp  8    TMA loads (one thread): Q once, then K and V tiles
 //   warp  9    MMA issue (one thread) and the TMEM allocation
-// TMEM (64 columns): S^T of warpgroup 0 | S^T of warpgroup 1 (16 columns
-// each) | O^T 0 | O^T 1. Shared memory: the Q tile (16 rows x d) and the two
-// P^T buffers (16 rows x 128 keys), K-major in the 128-byte swizzled layout,
+// TMEM (64 columns): S^T of each warpgroup (16 columns each), then O^T of
+// each. Shared memory: the Q tile (16 rows x d) and one P^T buffer per
+// warpgroup (16 rows x 128 keys), K-major in the 128-byte swizzled layout,
 // then a ring of K/V slots in the layout the forward kernel uses.
 //
-// Order of the products: QK(0) | QK(1) PV(0) | QK(2) PV(1) | ... | PV(n-1).
-// Every wait is bounded (Watchdog).
+// Order of the products: QK(0) | QK(1) PV(0) | QK(2) PV(1) | ... : the scores
+// of the next kDecAhead = kDecWG - 1 tiles are issued before each P.V, so
+// every warpgroup has a tile to work on. Every wait is bounded (Watchdog).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -61,9 +64,12 @@ namespace fa {
 
 constexpr int kDecCols = 16;        // N of both products: query columns of the tile
 constexpr int kDecLive = 8;         // live columns (G heads x Nq rows) the softmax handles
-constexpr int kDecThreads = 320;
-constexpr int kDecTmaWarp = 8;
-constexpr int kDecMmaWarp = 9;
+constexpr int kDecWG = 2;                    // softmax warpgroups, taking the key tiles in turn
+constexpr int kDecAhead = kDecWG - 1;        // key tiles whose scores are issued ahead of a P.V
+constexpr int kDecThreads = 32 * (4 * kDecWG + 2);
+constexpr int kDecTmaWarp = 4 * kDecWG;
+constexpr int kDecMmaWarp = 4 * kDecWG + 1;
+static_assert(kDecWG >= 2 && kDecWG <= 3, "two or three softmax warpgroups");
 
 // E: bytes per element of Q, K, V and P (2: bf16; 1: e4m3 with kind::f8f6f4
 // products, P rounded to e4m3).
@@ -80,11 +86,11 @@ struct DecCfg {
     static constexpr int kQBytes = kBlocks * kColBlockBytes;
     static constexpr int kPBytes = (kTile * E / 128) * kColBlockBytes;   // 16 x 128 keys
     static constexpr int kSlots = E == 2 ? 6 : 12;           // K/V ring depth
-    static constexpr int kSmemTiles = kQBytes + 2 * kPBytes + kSlots * kTileBytes;
+    static constexpr int kSmemTiles = kQBytes + kDecWG * kPBytes + kSlots * kTileBytes;
     static constexpr int kSmemBytes = kSmemTiles + 1024 /*alignment*/ + 4096 /*barriers*/;
-    static constexpr uint32_t kTmemCols = 64;
+    static constexpr uint32_t kTmemCols = 2 * kDecWG * kDecCols <= 64 ? 64 : 128;
     static constexpr uint32_t col_s(int w) { return (uint32_t)(w * kDecCols); }
-    static constexpr uint32_t col_o(int w) { return (uint32_t)((2 + w) * kDecCols); }
+    static constexpr uint32_t col_o(int w) { return (uint32_t)((kDecWG + w) * kDecCols); }
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
     static_assert(kSlots <= 12, "K/V ring barriers");
 };
@@ -93,21 +99,22 @@ struct DecBarriers {
     uint64_t q_full;
     uint64_t kv_full[12];
     uint64_t kv_empty[12];
-    // per warpgroup w (= key-tile parity)
-    uint64_t s_full[2];       // S^T of a key tile is in TMEM (MMA commit)
-    uint64_t s_free[2];       // its 128 threads have read it (128 arrivals)
-    uint64_t p_full[2];       // P^T in shared memory (128 arrivals)
-    uint64_t p_free[2];       // P.V has read it (MMA commit)
-    uint64_t pv_done[2];      // one phase per P.V product of the warpgroup
-    uint64_t red_full[2][2];  // [w][tile parity within w]: column maxima (128 arrivals)
-    uint64_t sum_full[2];     // column sums, epilogue (128 arrivals)
-    uint64_t merge_full;      // warpgroup 1's column (m, l, lr) for warpgroup 0 (128)
+    // per warpgroup w (key tiles j with j % kDecWG == w)
+    uint64_t s_full[kDecWG];       // S^T of a key tile is in TMEM (MMA commit)
+    uint64_t s_free[kDecWG];       // its 128 threads have read it (128 arrivals)
+    uint64_t p_full[kDecWG];       // P^T in shared memory (128 arrivals)
+    uint64_t p_free[kDecWG];       // P.V has read it (MMA commit)
+    uint64_t pv_done[kDecWG];      // one phase per P.V product of the warpgroup
+    uint64_t red_full[kDecWG][2];  // [w][tile parity within w]: column maxima (128 arrivals)
+    uint64_t sum_full[kDecWG];     // column sums, epilogue (128 arrivals)
+    uint64_t merge_full;           // the other warpgroups' column (m, l, lr) for warpgroup 0
     uint64_t o_final;         // every product of the unit has completed
     uint64_t teardown;
-    float red[2][2][4][kDecLive];
-    float sum_l[2][4][kDecLive];
-    float sum_lr[2][4][kDecLive];
-    float merge_m[kDecLive], merge_l[kDecLive], merge_lr[kDecLive];
+    float red[kDecWG][2][4][kDecLive];
+    float sum_l[kDecWG][4][kDecLive];
+    float sum_lr[kDecWG][4][kDecLive];
+    float merge_m[kDecWG - 1][kDecLive], merge_l[kDecWG - 1][kDecLive],
+        merge_lr[kDecWG - 1][kDecLive];
     uint32_t tmem_base;
     int abort;
     int skip;
@@ -166,7 +173,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sP = sQ + C::kQBytes;                          // one buffer per warpgroup
-    uint8_t* sKV = sP + 2 * C::kPBytes;
+    uint8_t* sKV = sP + kDecWG * C::kPBytes;
     DecBarriers* bars = reinterpret_cast<DecBarriers*>(smem + C::kSmemTiles);
 
     // ---------------------------------------------------------- the unit
@@ -193,7 +200,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             mbar_init(&bars->kv_full[s], 1);
             mbar_init(&bars->kv_empty[s], 1);
         }
-        for (int w = 0; w < 2; ++w) {
+        for (int w = 0; w < kDecWG; ++w) {
             mbar_init(&bars->s_full[w], 1);
             mbar_init(&bars->s_free[w], kTile);
             mbar_init(&bars->p_full[w], kTile);
@@ -203,7 +210,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             mbar_init(&bars->red_full[w][1], kTile);
             mbar_init(&bars->sum_full[w], kTile);
         }
-        mbar_init(&bars->merge_full, kTile);
+        mbar_init(&bars->merge_full, kTile * (kDecWG - 1));
         mbar_init(&bars->o_final, 1);
         mbar_init(&bars->teardown, 1);
         bars->abort = 0;
@@ -213,7 +220,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // Q rows past the live columns are never loaded and P^T rows past kDecLive
     // never written: zero both once, so the padding columns of S^T are finite
     // (and masked) and those of O^T stay 0.
-    for (int e = tid; e < (C::kQBytes + 2 * C::kPBytes) / 16; e += kDecThreads)
+    for (int e = tid; e < (C::kQBytes + kDecWG * C::kPBytes) / 16; e += kDecThreads)
         reinterpret_cast<uint4*>(sQ)[e] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     if (warp == kDecMmaWarp) {
@@ -256,23 +263,26 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             for (int blk = 0; blk < C::kBlocks; ++blk)
                 tma_load_3d(&tm_q, &bars->q_full, sQ + blk * C::kColBlockBytes, blk * C::kBlockElems, 0,
                             b * p.H + h0);
-            // Loads in the order the MMAs consume them: K0 | K1 V0 | K2 V1 | ... | V(n-1).
-            const int loads = 2 * n;
+            // Loads in the order the MMAs consume them (see the MMA issuer):
+            // K(0) .. K(kDecAhead - 1), then K(i + kDecAhead) and V(i) for each i.
             int issued = 0;
-            for (int c = 0; ok && c < loads; ++c) {
-                const bool is_v = (c > 0) && ((c & 1) == 0 || (c + 1) / 2 >= n);
-                const int tile = (c == 0) ? 0 : is_v ? ((c & 1) ? n - 1 : c / 2 - 1) : (c + 1) / 2;
-                const int slot = c % C::kSlots;
-                const uint32_t round = (uint32_t)(c / C::kSlots);
-                ok = mbar_wait(&bars->kv_empty[slot], (round & 1u) ^ 1u, wd);
-                if (!ok) break;
+            auto load = [&](bool is_v, int tile) -> bool {
+                const int slot = issued % C::kSlots;
+                const uint32_t round = (uint32_t)(issued / C::kSlots);
+                if (!mbar_wait(&bars->kv_empty[slot], (round & 1u) ^ 1u, wd)) return false;
                 uint8_t* dst = sKV + slot * C::kTileBytes;
                 mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
                 for (int blk = 0; blk < C::kBlocks; ++blk)
                     tma_load_3d_hint(is_v ? &tm_v : &tm_k, &bars->kv_full[slot],
-                                     dst + blk * C::kBlockBytes, blk * C::kBlockElems, (kt0 + tile) * kTile,
-                                     bkv, pol_kv);
+                                     dst + blk * C::kBlockBytes, blk * C::kBlockElems,
+                                     (kt0 + tile) * kTile, bkv, pol_kv);
                 ++issued;
+                return true;
+            };
+            for (int j = 0; ok && j < min(kDecAhead, n); ++j) ok = load(false, j);
+            for (int i = 0; ok && i < n; ++i) {
+                if (i + kDecAhead < n) ok = load(false, i + kDecAhead);
+                if (ok) ok = load(true, i);
             }
             // Drain: every copy issued must land before the CTA exits.
             for (int c = max(0, issued - C::kSlots); c < issued; ++c)
@@ -298,50 +308,58 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
             constexpr uint64_t kPStep = (uint64_t)(C::kPBytes >> 4);
             bool ok = mbar_wait(&bars->q_full, 0u, wd);
-            int c = 0;
-            for (int j = 0; ok && j <= n; ++j) {
-                if (j < n) {
-                    // S^T(j) = K(j) . Q^T into warpgroup (j & 1)'s buffer, once it
-                    // has read its previous tile j - 2 there
-                    const int w = j & 1;
-                    const int slot = c % C::kSlots;
-                    ok = mbar_wait(&bars->kv_full[slot], (uint32_t)(c / C::kSlots) & 1u, wd);
-                    if (ok && j >= 2)
-                        ok = mbar_wait(&bars->s_free[w], (uint32_t)((j >> 1) - 1) & 1u, wd);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t a = dk0 + (uint64_t)slot * kTileStep;
+            int c = 0;   // K/V loads consumed, in the producer's order
+            // S^T(j) = K(j) . Q^T into warpgroup (j % kDecWG)'s buffer, once it
+            // has read its previous tile there
+            auto issue_qk = [&](int j) -> bool {
+                const int w = j % kDecWG;
+                const int slot = c % C::kSlots;
+                if (!mbar_wait(&bars->kv_full[slot], (uint32_t)(c / C::kSlots) & 1u, wd)) return false;
+                if (j >= kDecWG &&
+                    !mbar_wait(&bars->s_free[w], (uint32_t)(j / kDecWG - 1) & 1u, wd))
+                    return false;
+                tc_fence_after();
+                const uint64_t a = dk0 + (uint64_t)slot * kTileStep;
 #pragma unroll
-                    for (int kk = 0; kk < D * E / 32; ++kk) {       // 32-byte K-steps
-                        const uint64_t oa = (uint64_t)(((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4);
-                        const uint64_t ob = (uint64_t)(((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4);
-                        mma(tmem + C::col_s(w), a + oa, dq + ob, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&bars->s_full[w]);
-                    umma_commit(&bars->kv_empty[slot]);
-                    ++c;
+                for (int kk = 0; kk < D * E / 32; ++kk) {       // 32-byte K-steps
+                    const uint64_t oa = (uint64_t)(((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4);
+                    const uint64_t ob = (uint64_t)(((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4);
+                    mma(tmem + C::col_s(w), a + oa, dq + ob, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                if (j >= 1) {
-                    // O^T(w) += V(jj)^T . P^T(jj), w = jj & 1
-                    const int jj = j - 1, w = jj & 1;
-                    const int slot = c % C::kSlots;
-                    ok = mbar_wait(&bars->kv_full[slot], (uint32_t)(c / C::kSlots) & 1u, wd);
-                    if (ok) ok = mbar_wait(&bars->p_full[w], (uint32_t)(jj >> 1) & 1u, wd);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t a = dv0 + (uint64_t)slot * kTileStep;
-                    const uint64_t bp = dp0 + (uint64_t)w * kPStep;
+                umma_commit(&bars->s_full[w]);
+                umma_commit(&bars->kv_empty[slot]);
+                ++c;
+                return true;
+            };
+            // O^T(w) += V(j)^T . P^T(j), w = j % kDecWG
+            auto issue_pv = [&](int j) -> bool {
+                const int w = j % kDecWG;
+                const int slot = c % C::kSlots;
+                if (!mbar_wait(&bars->kv_full[slot], (uint32_t)(c / C::kSlots) & 1u, wd)) return false;
+                if (!mbar_wait(&bars->p_full[w], (uint32_t)(j / kDecWG) & 1u, wd)) return false;
+                tc_fence_after();
+                const uint64_t a = dv0 + (uint64_t)slot * kTileStep;
+                const uint64_t bp = dp0 + (uint64_t)w * kPStep;
 #pragma unroll
-                    for (int kk = 0; kk < kTile * E / 32; ++kk) {   // 32 / E keys per K-step
-                        const uint64_t oa = (uint64_t)((kk * (32 / E) * 128) >> 4);
-                        const uint64_t ob = (uint64_t)(((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4);
-                        mma(tmem + C::col_o(w), a + oa, bp + ob, idesc_o, (jj > 1 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&bars->pv_done[w]);
-                    umma_commit(&bars->p_free[w]);
-                    umma_commit(&bars->kv_empty[slot]);
-                    ++c;
+                for (int kk = 0; kk < kTile * E / 32; ++kk) {   // 32 / E keys per K-step
+                    const uint64_t oa = (uint64_t)((kk * (32 / E) * 128) >> 4);
+                    const uint64_t ob = (uint64_t)(((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4);
+                    mma(tmem + C::col_o(w), a + oa, bp + ob, idesc_o,
+                        (j >= kDecWG || kk > 0) ? 1u : 0u);
                 }
+                umma_commit(&bars->pv_done[w]);
+                umma_commit(&bars->p_free[w]);
+                umma_commit(&bars->kv_empty[slot]);
+                ++c;
+                return true;
+            };
+            // QK(0) .. QK(kDecAhead - 1) | QK(i + kDecAhead) PV(i) | ...: while P.V(i)
+            // waits for its probabilities, the scores of the next kDecAhead tiles are
+            // in flight, one per other warpgroup.
+            for (int j = 0; ok && j < min(kDecAhead, n); ++j) ok = issue_qk(j);
+            for (int i = 0; ok && i < n; ++i) {
+                if (i + kDecAhead < n) ok = issue_qk(i + kDecAhead);
+                if (ok) ok = issue_pv(i);
             }
             umma_commit(&bars->o_final);
             // Drain: all MMAs issued by this thread complete before teardown.
@@ -350,8 +368,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         __syncwarp();
     } else {
-        // ====================================================== softmax (warps 0-7)
-        const int wg = warp >> 2;                           // warpgroup = key-tile parity
+        // ====================================================== softmax (warps 0 .. 4 kDecWG - 1)
+        const int wg = warp >> 2;                           // warpgroup: key tiles j % kDecWG == wg
         const int wq = warp & 3;                            // warp within the warpgroup
         const int t = tid & (kTile - 1);                    // key of a tile / head-dim index
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
@@ -364,8 +382,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             lr[q] = 0.f;
         }
         bool ok = true;
-        for (int j = wg; j < n; j += 2) {
-            const int jo = j >> 1;                          // index among this warpgroup's tiles
+        for (int j = wg; j < n; j += kDecWG) {
+            const int jo = j / kDecWG;                      // index among this warpgroup's tiles
             const int rb = jo & 1;                          // maxima buffer
             ok = mbar_wait(&bars->s_full[wg], (uint32_t)jo & 1u, wd);
             ok = __all_sync(0xffffffffu, ok);
@@ -409,7 +427,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
             if (rescale) {   // uniform in the warpgroup: every thread sees the same maxima
                 // O^T(wg) holds the products of this warpgroup's tiles < j; the
-                // last of them, P.V(j - 2), was issued before Q.K^T(j), whose
+                // last of them, P.V(j - kDecWG), was issued before Q.K^T(j), whose
                 // scores are in, so pv_done is exactly at that phase. Then each
                 // column that moves is scaled; thread t holds head-dim row t.
                 ok = mbar_wait(&bars->pv_done[wg], (uint32_t)(jo - 1) & 1u, wd);
@@ -435,7 +453,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
 
             // probabilities of this key, rounded to bf16 (e4m3) into the warpgroup's P^T
-            if (jo >= 1) {   // P.V(j - 2) has read the buffer (complete, as above)
+            if (jo >= 1) {   // P.V(j - kDecWG) has read the buffer (complete, as above)
                 ok = mbar_wait(&bars->p_free[wg], (uint32_t)(jo - 1) & 1u, wd);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -473,9 +491,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
 
         // ------------------------------------------------ epilogue
-        // Each warpgroup sums its columns over its 128 key threads; warpgroup 1
-        // hands (m_ref, l, lr) to warpgroup 0, which merges the two halves and
-        // writes the rows (thread t: head-dim index t).
+        // Each warpgroup sums its columns over its 128 key threads; the others
+        // hand (m_ref, l, lr) to warpgroup 0, which merges the kDecWG parts by
+        // their log-sum-exp and writes the rows (thread t: head-dim index t).
         if (ok) {
             ok = mbar_wait(&bars->o_final, 0u, wd);
             ok = __all_sync(0xffffffffu, ok);
@@ -501,13 +519,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                    bars->sum_lr[wg][3][q];
         };
         if (ok) {
-            if (wg == 1) {
+            if (wg > 0) {
 #pragma unroll
                 for (int q = 0; q < kDecLive; ++q)
                     if (q == t) {
-                        bars->merge_m[q] = m_ref[q];
-                        bars->merge_l[q] = col_l(q);
-                        bars->merge_lr[q] = col_lr(q);
+                        bars->merge_m[wg - 1][q] = m_ref[q];
+                        bars->merge_l[wg - 1][q] = col_l(q);
+                        bars->merge_lr[wg - 1][q] = col_lr(q);
                     }
                 mbar_arrive(&bars->merge_full);
             } else {
@@ -517,27 +535,39 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         if (ok && wg == 0) {
             tc_fence_after();
-            uint32_t o0[kDecLive], o1[kDecLive];
-            if (n > 0) tmem_ld8(tmem + lane_base + C::col_o(0), o0);
-            if (n > 1) tmem_ld8(tmem + lane_base + C::col_o(1), o1);
+            uint32_t o[kDecWG][kDecLive];
+#pragma unroll
+            for (int w = 0; w < kDecWG; ++w)
+                if (n > w) tmem_ld8(tmem + lane_base + C::col_o(w), o[w]);
             tmem_wait_ld();
             const bool part = p.o_part != nullptr;
             const size_t rows = (size_t)p.B * p.H * Nq;
 #pragma unroll
             for (int q = 0; q < kDecLive; ++q) {
                 if (q >= cols) break;
-                const float m1 = bars->merge_m[q], l1 = bars->merge_l[q], lr1 = bars->merge_lr[q];
-                const float m0 = m_ref[q], l0 = col_l(q), lr0 = col_lr(q);
-                // weights of the two halves (a half with no visible key weighs 0
-                // and its accumulator, possibly never written, is not read)
-                const float mm = fmaxf(l0 > 0.f ? m0 : -INFINITY, l1 > 0.f ? m1 : -INFINITY);
-                const float a0 = (l0 > 0.f) ? fast_exp2((m0 - mm) * c) : 0.f;
-                const float a1 = (l1 > 0.f) ? fast_exp2((m1 - mm) * c) : 0.f;
-                const float lsum = l0 * a0 + l1 * a1;
-                const float lrsum = lr0 * a0 + lr1 * a1;
-                float acc = 0.f;
-                if (a0 > 0.f) acc += __uint_as_float(o0[q]) * a0;
-                if (a1 > 0.f) acc += __uint_as_float(o1[q]) * a1;
+                float mw[kDecWG], lw[kDecWG], lrw[kDecWG];
+                mw[0] = m_ref[q];
+                lw[0] = col_l(q);
+                lrw[0] = col_lr(q);
+#pragma unroll
+                for (int w = 1; w < kDecWG; ++w) {
+                    mw[w] = bars->merge_m[w - 1][q];
+                    lw[w] = bars->merge_l[w - 1][q];
+                    lrw[w] = bars->merge_lr[w - 1][q];
+                }
+                // weights of the parts (a part with no visible key weighs 0 and
+                // its accumulator, possibly never written, is not read)
+                float mm = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kDecWG; ++w) mm = fmaxf(mm, lw[w] > 0.f ? mw[w] : -INFINITY);
+                float lsum = 0.f, lrsum = 0.f, acc = 0.f;
+#pragma unroll
+                for (int w = 0; w < kDecWG; ++w) {
+                    const float aw = (lw[w] > 0.f) ? fast_exp2((mw[w] - mm) * c) : 0.f;
+                    lsum += lw[w] * aw;
+                    lrsum += lrw[w] * aw;
+                    if (aw > 0.f) acc += __uint_as_float(o[w][q]) * aw;
+                }
                 const int g = q / Nq, rr = q - g * Nq;
                 const size_t row = (size_t)(b * p.H + h0 + g) * Nq + rr;
                 // a column with no visible key: O = 0, lse = -inf
