@@ -33,7 +33,7 @@ def fa():
     return fa
 
 
-def run_fp8(fa, q8, k8, v8, sc, causal, kv_len=None, cache=False, splits=None):
+def run_fp8(fa, q8, k8, v8, sc, causal, kv_len=None, cache=False, splits=None, scale=None):
     """One e4m3 launch: square (fa_fwd_fp8) or, with cache=True, through the
     split-KV entry (Nq <= Nk, query heads of a K/V group packed)."""
     dev = torch.device("cuda:0")
@@ -43,10 +43,11 @@ def run_fp8(fa, q8, k8, v8, sc, causal, kv_len=None, cache=False, splits=None):
     out = torch.full((B, H, N, d), float("nan"), dtype=torch.bfloat16, device=dev)
     lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
     if cache:
-        fa.decode_attention_fp8(qd, kd, vd, *sc, causal=causal, kv_len=kvd,
+        fa.decode_attention_fp8(qd, kd, vd, *sc, scale=scale, causal=causal, kv_len=kvd,
                                 num_splits=splits, out=out, lse=lse)
     else:
-        fa.attention_fp8(qd, kd, vd, *sc, causal=causal, kv_len=kvd, out=out, lse=lse)
+        fa.attention_fp8(qd, kd, vd, *sc, scale=scale, causal=causal, kv_len=kvd, out=out,
+                         lse=lse)
     st = fa.fa_last_device_error(torch.cuda.current_stream().cuda_stream)
     assert st == fa.FA_OK, fa.fa_status_string(st)
     return out.double().cpu().numpy(), lse.double().cpu().numpy()
@@ -200,3 +201,31 @@ def test_fp8_head_dim_64_grouped_heads_padding_and_cache(fa, causal):
         check_fp8(fa, 2, 8, 2, 5, causal, seed=6960 + causal, d=64, Nk=2000, splits=splits)
         check_fp8(fa, 1, 4, 4, 200, causal, seed=6970 + causal, d=64, Nk=1000, splits=splits)
 
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_fp8_reference_moves_square(fa, d):
+    """e4m3 scores that climb tile by tile at different rates within a warp.
+    Query row i carries a_i in {0, 1/8, 1/2, 1} (cycling) in column 0, key j
+    carries 48 * (j // 128) there (exact in e4m3 up to 288), the other columns
+    small values; with scale 1/8 a key tile raises a row's scores by 8.66 a_i
+    log2 units, so rows with a_i = 1 move their reference maximum (threshold 8)
+    on every later tile, a_i = 1/2 every other tile, the rest never. Without
+    the moves, tile 6's probabilities for a_i = 1 would be 2^52 and saturate at
+    448, so O within the e4m3 bound shows the rescale of O and l ran."""
+    N, scale = 7 * 128, 0.125
+    g = torch.Generator().manual_seed(5)
+    q = 0.25 * torch.randn(1, 2, N, d, generator=g)
+    k = 0.25 * torch.randn(1, 2, N, d, generator=g)
+    v = torch.randn(1, 2, N, d, generator=g)
+    q[..., 0] = torch.tensor([0.0, 0.125, 0.5, 1.0]).repeat(N // 4)
+    k[..., 0] = 48.0 * (torch.arange(N) // 128).float()
+    q8, k8, v8 = (x.to(torch.float8_e4m3fn) for x in (q, k, v))
+    assert torch.equal(k8[0, 0, :, 0].float(), 48.0 * (torch.arange(N) // 128).float())
+    assert 48 * scale * math.log2(math.e) > 8
+    sc = (1.0, 1.0, 1.0)
+    vmax = float(np.abs(ofp8.decode_e4m3(v8.view(torch.uint8).numpy())).max())
+    for causal in (False, True):
+        o, lse = run_fp8(fa, q8, k8, v8, sc, causal, scale=scale)
+        o_ref, lse_ref = ofp8.attention_fp8(q8, k8, v8, *sc, scale, causal=causal)
+        compare_fp8(o, lse, o_ref, lse_ref, vmax, f"e4m3 climbing scores d={d} causal={causal}")
