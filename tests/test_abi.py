@@ -268,3 +268,19 @@ def test_fp8_splitkv_argument_errors_are_synchronous(lib, over, status):
                                 a["ws_bytes"], None)
     assert st == status
 
+
+
+def test_default_splits_rule(lib):
+    """fa_splitkv_default_splits keeps units within one wave: at most 128 units
+    for shapes the decoding tile takes (d = 128, query heads per K/V head x rows
+    <= 8), at most the SM count otherwise (148 here: with no device the count
+    falls back to 148), and each range at least four key tiles long."""
+    f = lib.fa_splitkv_default_splits
+    assert f(1, 32, 8, 1, 131072, 128) == 16        # 8 head groups x 16 = 128 units
+    assert f(2, 32, 8, 1, 65536, 128) == 8          # 16 x 8 = 128
+    assert f(4, 32, 8, 1, 32768, 128) == 4          # 32 x 4 = 128
+    assert f(16, 32, 8, 1, 8192, 128) == 1          # 128 units unsplit
+    assert f(1, 32, 8, 1, 131072, 64) == 18         # general kernel: 8 x 18 = 144 <= 148
+    assert f(1, 32, 2, 1, 131072, 128) == 74        # 16 heads per group: general kernel, 2 x 74
+    assert f(1, 32, 8, 1, 1024, 128) == 2           # 8 key tiles: ranges of >= 4 tiles
+    assert f(1, 32, 7, 1, 4096, 128) == 1           # H not a multiple of H_kv: invalid, 1
